@@ -1,0 +1,185 @@
+/*
+ * rolaq.h — C ABI of librolaq.so: a 2-bit rotated MLA latent cache on B200 (sm_100a).
+ *
+ * Method: "RoLaQ: Joint Rotation and Range Calibration for 2-Bit KV Caches in
+ * Multi-Head Latent Attention" (arXiv 2610.20686v1).  Passages cited below by
+ * page title and section:
+ *   [S2.1]  §2.1 "One Cache, Two Roles": one content latent feeds K and V; the 64-d
+ *           RoPE key k_R stays in BF16.
+ *   [S3.2]  §3.2 "Response-Preserving Range Calibration": a per-layer threshold tau
+ *           assigns standardized coordinates to four levels; the gain g scales the
+ *           reconstruction around the group mean.
+ *   [S3.3]  §3.3 "Joint Calibration and Inference": serving stores rotated latents as
+ *           2-bit codes and folds the read-side rotation into the absorbed projections.
+ *   [S4.1]  §4.1 "Setup": protection keeps the first 4 sink and the most recent tokens
+ *           in BF16.
+ *   [A.3]   §A.3 "Calibration and Storage": 288 B per unprotected token per layer
+ *           (packed codes + group statistics + BF16 RoPE key); protected tokens also
+ *           store BF16 content.
+ *   [NB]    "2610.20686-rolaq-cache-accounting" notebook: 128 B of 2-bit codes +
+ *           32 B of FP32 group statistics (two per 128-coordinate group) + 128 B BF16
+ *           RoPE key = 288 B, versus 1152 B for BF16 MLA (4.000x ceiling).
+ *
+ * Conventions for every entry point:
+ *   - All pointers named *_dev are device pointers owned by the caller; the library
+ *     never allocates, frees or keeps them.  Host pointers are read during the call only.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; the call returns once the kernels are launched.
+ *   - Return value: ROLAQ_OK (0) or a negative ROLAQ_E* code.  Argument errors are
+ *     detected on the host before anything is launched.  Errors that only the device can
+ *     see (a page-table entry outside the pool) set bits in a device status word, skip
+ *     the offending access and never trap; read them with rolaq_get_status().
+ *   - bf16 means IEEE bfloat16 stored as uint16_t.
+ */
+#ifndef ROLAQ_H_
+#define ROLAQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- fixed shapes [S2.1], [A.3], [NB] ------------------------------------------- */
+#define ROLAQ_D_C          512   /* content-latent width                              */
+#define ROLAQ_D_R          64    /* RoPE-key width                                    */
+#define ROLAQ_GROUP        128   /* coordinates per quantization group                */
+#define ROLAQ_GROUPS       4     /* groups per token = D_C / GROUP                    */
+#define ROLAQ_CODE_BYTES   128   /* 512 coordinates x 2 bit                           */
+#define ROLAQ_META_BYTES   32    /* 4 groups x (mean, scale) fp32                     */
+#define ROLAQ_KR_BYTES     128   /* 64 x bf16                                         */
+#define ROLAQ_TOKEN_BYTES  288   /* CODE + META + KR                                  */
+#define ROLAQ_BF16_TOKEN_BYTES 1152 /* (512 + 64) x bf16, the uncompressed MLA record */
+
+/* ---- page layout ---------------------------------------------------------------
+ * The cache is a pool of fixed-size pages.  A page holds ROLAQ_PAGE_TOKENS tokens of
+ * one request as three planes (structure of arrays inside the page):
+ *
+ *   offset     0: codes [64 tokens][128 B]   byte b of a token holds coordinates
+ *                                            4b..4b+3; coordinate j sits in bits
+ *                                            2*(j%4)..2*(j%4)+1.  Code values 0..3 mean
+ *                                            z < -tau, -tau <= z < 0, 0 <= z < tau,
+ *                                            z >= tau (ascending level order).
+ *   offset  8192: meta  [64 tokens][4 groups][2] fp32: (group mean, gain * group std)
+ *   offset 10240: k_R   [64 tokens][64] bf16
+ *
+ * ROLAQ_PAGE_BYTES = 64 * 288 = 18432 = 144 rows of 128 B.  Token at logical position p
+ * of request r lives in page page_table[r * max_pages_per_seq + p / 64] at row p % 64.
+ * The pool base must be 1024-byte aligned (the decode kernel stages whole pages with
+ * a 128-byte-swizzled tensor copy).
+ * ------------------------------------------------------------------------------- */
+#define ROLAQ_PAGE_TOKENS  64
+#define ROLAQ_PAGE_BYTES   18432
+#define ROLAQ_PAGE_CODES_OFFSET 0
+#define ROLAQ_PAGE_META_OFFSET  8192
+#define ROLAQ_PAGE_KR_OFFSET    10240
+
+/* Rotation operand prepared by rolaq_prepare_rotation: two bf16 planes [2][512][512]. */
+#define ROLAQ_RSPLIT_BYTES (2u * 512u * 512u * 2u)
+
+/* ---- error codes ---------------------------------------------------------------- */
+#define ROLAQ_OK            0
+#define ROLAQ_EINVAL       -1   /* null / misaligned pointer, bad size or shape        */
+#define ROLAQ_ENOSPACE     -2   /* workspace smaller than rolaq_decode_workspace_bytes */
+#define ROLAQ_ECUDA        -3   /* a CUDA runtime or driver call failed                */
+#define ROLAQ_EUNSUPPORTED -4   /* shape the kernels do not implement (heads % 16)     */
+
+/* Device status bits reported by rolaq_get_status(). */
+#define ROLAQ_STATUS_BAD_PAGE   1  /* page-table entry < 0 or >= num_pages (skipped)  */
+#define ROLAQ_STATUS_BAD_SLOT   2  /* append target outside its request's pages       */
+
+/* Cache descriptor.  Plain data; the caller owns every buffer it points to.
+ *   pages_dev       page pool, num_pages * ROLAQ_PAGE_BYTES bytes, 1024-B aligned.
+ *   page_table_dev  int32 [batch][max_pages_per_seq]; entry = page index in the pool.
+ *   prot_dev        optional BF16 side store [batch][n_sink + n_recent][512] holding the
+ *                   rotated content of protected tokens [S4.1], [A.3]; NULL when
+ *                   n_sink + n_recent == 0.  Row p (p < n_sink) holds sink position p;
+ *                   row n_sink + (p % n_recent) holds recent position p.               */
+typedef struct rolaq_cache {
+    void*          pages_dev;
+    int64_t        num_pages;
+    const int32_t* page_table_dev;
+    int32_t        batch;
+    int32_t        max_pages_per_seq;
+    void*          prot_dev;
+    int32_t        n_sink;
+    int32_t        n_recent;
+} rolaq_cache;
+
+/* Per-layer quantizer constants, fixed during serving [S3.3].
+ *   level_a, level_b: the four reconstruction levels are -b, -a, +a, +b, the centroids
+ *   of a standard normal on [0, tau) and [tau, inf) mirrored [S3.2].                 */
+typedef struct rolaq_layer_params {
+    float tau;
+    float gain;
+    float level_a;
+    float level_b;
+} rolaq_layer_params;
+
+/* Fill p for threshold tau > 0 and gain > 0.  The levels are computed on the host in
+ * double (a = (phi(0) - phi(tau)) / (Phi(tau) - 1/2), b = phi(tau) / (1 - Phi(tau)))
+ * and rounded to fp32 once.  Returns ROLAQ_EINVAL for a non-finite or non-positive
+ * tau or gain.  [S3.2]                                                                */
+int rolaq_layer_params_init(rolaq_layer_params* p, float tau, float gain);
+
+/* Convert the fp32 rotation R_dev [512][512] (row-major, y = c . R for a row vector c)
+ * into the tensor-core operand R_split_dev (ROLAQ_RSPLIT_BYTES, 16-B aligned): plane 0
+ * holds bf16(R^T), plane 1 holds bf16(R^T - plane0), both [512 out][512 in].  The pair
+ * reproduces R to about 2^-17 relative, so y keeps fp32-level accuracy.  Run once per
+ * layer at load time.  [S3.3]                                                         */
+int rolaq_prepare_rotation(const float* R_dev, void* R_split_dev, void* stream);
+
+/* Write path [S3.2], [S3.3], [A.3]: for each of n tokens i, rotate c_dev[i] (bf16 [n][512])
+ * by R, split into 4 groups of 128, standardise each group by its fp32 mean and
+ * population std, assign 2-bit codes by tau, pack, and store (mean, gain*std) and the
+ * bf16 RoPE key k_R_dev[i] ([n][64]) into the page of request req_dev[i] at logical
+ * position pos_dev[i].  With protection configured, the token's bf16 rotated content is
+ * also written to the side store when pos < n_sink (sink row) or
+ * pos >= seq_lens_dev[req] - n_recent (recent ring row), where seq_lens_dev (int32
+ * [batch], may be NULL when n_recent == 0) holds each request's length after this
+ * append.  A group with zero spread gets code 2 and scale 0.  Targets outside the page
+ * table set ROLAQ_STATUS_BAD_SLOT and are skipped.  n == 0 is a no-op.               */
+int rolaq_quantize_append(const rolaq_cache* cache, const rolaq_layer_params* p,
+                          const void* R_split_dev, const void* c_dev, const void* k_R_dev,
+                          const int32_t* req_dev, const int32_t* pos_dev,
+                          const int32_t* seq_lens_dev, int n, void* stream);
+
+/* Bytes of device workspace rolaq_decode_attn needs for `batch` requests and `heads`
+ * query heads on the current device (split-K partials and their merge state).          */
+size_t rolaq_decode_workspace_bytes(int batch, int heads);
+
+/* Read path [S2.1], [S3.3]: absorbed-MLA decode attention straight from the packed cache.
+ * For request r with L = seq_lens_dev[r] tokens and head h:
+ *   x_t      = mean_g + scale_g * level(code)      (2-bit token)  or the bf16 side-store
+ *              row (protected token: t < n_sink, or t >= L - n_recent)
+ *   s_t      = (q_c_rot[r,h] . x_t + q_R[r,h] . k_R_t) * sm_scale
+ *   out[r,h] = sum_t softmax(s)_t x_t                (rotated basis; the inverse rotation
+ *              belongs to the absorbed value projection [S3.3])
+ *   lse[r,h] = log sum_t exp(s_t)                    (natural log)
+ * q_c_rot_dev bf16 [batch][heads][512] already carries R (q . W_UK . R), q_R_dev bf16
+ * [batch][heads][64]; out_dev fp32 [batch][heads][512]; lse_dev fp32 [batch][heads]
+ * (may be NULL).  heads must be a positive multiple of 16, batch <= cache->batch.
+ * L == 0 gives out = 0 and lse = -inf.  workspace_dev (16-B aligned) must hold
+ * rolaq_decode_workspace_bytes(batch, heads) bytes; it is scratch owned by the caller
+ * and needs no initialisation.  Split-K over the sequence with a log-sum-exp merge.   */
+int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
+                      const void* q_c_rot_dev, const void* q_R_dev,
+                      const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
+                      float* out_dev, float* lse_dev,
+                      void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* Copy the device status word of the current device to *bits and clear it.  Blocks until
+ * `stream` has finished.                                                              */
+int rolaq_get_status(int* bits, void* stream);
+
+/* Static description of an error code. */
+const char* rolaq_strerror(int code);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int rolaq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* ROLAQ_H_ */
