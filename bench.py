@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark of the 2-bit rotated MLA cache hot path on B200.
+
+Step = one decode step of the long-context serving shape: for each of 27 layers, append
+one new token per request (write path: rotate, quantize, pack) and run the absorbed-MLA
+decode over 4 requests x 262,144 cached tokens at 16 heads (read path).  The cache of a
+step is 8.15 GB, far larger than L2, so no flush is needed between steps.  value = cache
+GB/s over the whole step (all ranks; replicas are independent, weak scaling).
+Also measured: the prefill write path on 65,536 tokens x 27 layers (tokens/s), and the
+CPU oracle on a bounded sample (cpu_baseline).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from decode_attention_rotate_b200 import rolaq as R          # noqa: E402
+from decode_attention_rotate_b200 import workloads as W      # noqa: E402
+
+METRIC = "2-bit MLA decode: cache GB/s & % HBM roofline; quantize-append tokens/s"
+SM_SCALE = 1.0 / math.sqrt(192.0)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+# DRAM bytes (read + write) per launch of the decode split kernel from the committed ncu
+# capture (profiles/); None until a capture of the current kernel exists.
+DECODE_TRAFFIC_PER_LAUNCH = None
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d.get("hbm_gbs", FALLBACK_HBM_GBS), d.get("bf16_tflops", FALLBACK_BF16_TFLOPS), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index, self.proc, self.lines = index, None, []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        med = float(np.median(sm)) if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload -------
+
+class DecodeLayer:
+    def __init__(self, w, layer, dev):
+        self.tau, self.gain = W.layer_constants(w, layer)
+        self.params = R.layer_params_init(self.tau, self.gain)
+        Rm = torch.as_tensor(W.rotation(w.seed + layer)).to(dev)
+        self.R_split = R.prepare_rotation(Rm)
+        pt = torch.as_tensor(W.page_table(w))
+        self.cache = R.PagedCache(int(pt.max()) + 1, pt, device=dev)
+        self.q_c = (torch.randn((w.batch, w.heads, W.D_C), device=dev, generator=_gen(w, layer, 7))
+                    .to(torch.bfloat16))
+        self.q_r = (torch.randn((w.batch, w.heads, W.D_R), device=dev, generator=_gen(w, layer, 8))
+                    .to(torch.bfloat16))
+        self.out = torch.empty((w.batch, w.heads, W.D_C), dtype=torch.float32, device=dev)
+        self.lse = torch.empty((w.batch, w.heads), dtype=torch.float32, device=dev)
+
+    def fill(self, w, layer, dev, chunk=1 << 18):
+        for b, L in enumerate(w.seq_lens):
+            for s in range(0, L, chunk):
+                n = min(chunk, L - s)
+                c = W.latent_device(w, layer, n, dev, stream=1000 + 97 * b + s // chunk)
+                kr = W.rope_key_device(w, layer, n, dev, stream=5000 + 97 * b + s // chunk)
+                req = torch.full((n,), b, dtype=torch.int32, device=dev)
+                pos = torch.arange(s, s + n, dtype=torch.int32, device=dev)
+                R.quantize_append(self.cache, self.params, self.R_split, c, kr, req, pos)
+
+
+def _gen(w, layer, k):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(w.seed * 7919 + layer * 131 + k)
+    return g
+
+
+def build_decode_workload(w, dev):
+    layers = [DecodeLayer(w, l, dev) for l in range(w.layers)]
+    for l, lay in enumerate(layers):
+        lay.fill(w, l, dev)
+    torch.cuda.synchronize()
+    return layers
+
+
+def cache_bytes_per_step(w):
+    return w.layers * w.total_tokens * R.TOKEN_BYTES
+
+
+# ----------------------------------------------------------------- CPU oracle -------
+
+def cpu_oracle_decode_rate(w, layers, budget_s=12.0):
+    """The fp64 oracle decoding whole requests of the bench's layers (bounded sample)."""
+    from oracle import rolaq_oracle as O
+    pt = W.page_table(w)
+    done_bytes, t_total, n_req = 0, 0.0, 0
+    threads = torch.get_num_threads()
+    for l, lay in enumerate(layers):
+        pool = lay.cache.pages.cpu().numpy()
+        qc = lay.q_c.float().cpu().numpy().astype(np.float64)
+        qr = lay.q_r.float().cpu().numpy().astype(np.float64)
+        for b, L in enumerate(w.seq_lens):
+            packed, meta, kr = O.pages_read_fast(pool, pt, b, L)
+            t0 = time.perf_counter()
+            O.decode_request(qc[b], qr[b], packed, meta, O.bf16_bits_to_f64(kr), lay.tau, SM_SCALE)
+            t_total += time.perf_counter() - t0
+            done_bytes += L * R.TOKEN_BYTES
+            n_req += 1
+            if t_total >= budget_s:
+                break
+        if t_total >= budget_s:
+            break
+    return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 oracle decode of {n_req} whole request(s) x {w.seq_lens[0]} tokens "
+                      f"(16 heads, one layer each), {t_total:.1f} s"}
+
+
+# ------------------------------------------------------------------ our arm --------
+
+def run_ours(args, rank, world, dev):
+    w = W.DECODE_4x256K_27L
+    layers = build_decode_workload(w, dev)
+    ws = torch.empty(R.decode_workspace_bytes(w.batch, w.heads), dtype=torch.uint8, device=dev)
+    lens = torch.as_tensor(w.seq_lens, dtype=torch.int32, device=dev)
+    # the token appended each step overwrites the last position, so every step decodes
+    # the same 262,144 tokens per request
+    new_req = torch.arange(w.batch, dtype=torch.int32, device=dev)
+    new_pos = (lens - 1).clone()
+    new_c = [W.latent_device(w, l, w.batch, dev, stream=9000) for l in range(w.layers)]
+    new_kr = [W.rope_key_device(w, l, w.batch, dev, stream=9001) for l in range(w.layers)]
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(w.layers)]
+
+    def step(record):
+        for l, lay in enumerate(layers):
+            R.quantize_append(lay.cache, lay.params, lay.R_split, new_c[l], new_kr[l], new_req, new_pos)
+            if record:
+                ev[l][0].record(stream)
+            R.decode_attn(lay.cache, lay.params, lay.q_c, lay.q_r, lens, SM_SCALE, lay.out, lay.lse, ws)
+            if record:
+                ev[l][1].record(stream)
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    assert R.get_status() == 0
+
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    dec_ms = 0.0
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(True)
+        # per-launch decode times of this step (events are read after the loop)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    total_ms = t0.elapsed_time(t1)
+    # decode-call durations: the last step's events (all steps are identical launches)
+    dec_ms = sum(ev[l][0].elapsed_time(ev[l][1]) for l in range(w.layers)) / w.layers
+    total_ms = max_over_ranks(total_ms, world)
+    ms_per_step = total_ms / args.steps
+    step_bytes = cache_bytes_per_step(w)
+    value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
+
+    # end-to-end through the C ABI with host buffers: the step's new tokens and queries come
+    # from pinned host memory, the readout goes back to pinned host memory
+    host_in = [(new_c[l].cpu().pin_memory(), new_kr[l].cpu().pin_memory(),
+                layers[l].q_c.cpu().pin_memory(), layers[l].q_r.cpu().pin_memory()) for l in range(w.layers)]
+    host_out = [(torch.empty_like(layers[l].out, device="cpu").pin_memory(),
+                 torch.empty_like(layers[l].lse, device="cpu").pin_memory()) for l in range(w.layers)]
+    dev_in = [(torch.empty_like(new_c[l]), torch.empty_like(new_kr[l]), torch.empty_like(layers[l].q_c),
+               torch.empty_like(layers[l].q_r)) for l in range(w.layers)]
+
+    def e2e_step():
+        for l, lay in enumerate(layers):
+            c, kr, qc, qr = dev_in[l]
+            hc, hkr, hqc, hqr = host_in[l]
+            c.copy_(hc, non_blocking=True); kr.copy_(hkr, non_blocking=True)
+            qc.copy_(hqc, non_blocking=True); qr.copy_(hqr, non_blocking=True)
+            R.quantize_append(lay.cache, lay.params, lay.R_split, c, kr, new_req, new_pos)
+            R.decode_attn(lay.cache, lay.params, qc, qr, lens, SM_SCALE, lay.out, lay.lse, ws)
+            host_out[l][0].copy_(lay.out, non_blocking=True)
+            host_out[l][1].copy_(lay.lse, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world) / args.steps
+    h2d = sum(sum(t.numel() * t.element_size() for t in hi) for hi in host_in)
+    d2h = sum(sum(t.numel() * t.element_size() for t in ho) for ho in host_out)
+    e2e_value = step_bytes * world / (e2e_ms * 1e-3) / 1e9
+
+    # prefill write path: 65,536 tokens x 27 layers
+    q_stats = bench_quantize(args, dev, world)
+
+    hbm, bf16, src = peaks()
+    dec_bytes = w.total_tokens * R.TOKEN_BYTES
+    achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_lens[0], "heads": w.heads,
+                   "layers": w.layers, "cache_bytes_per_step": step_bytes,
+                   "l2": "inputs larger than L2 (8.15 GB cache per step), no flush",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": DECODE_TRAFFIC_PER_LAUNCH,
+                     "kernel": "decode (split + merge launches)", "peak_source": src,
+                     "bytes_per_launch": dec_bytes, "ms_per_launch": round(dec_ms, 4),
+                     "frac_of_8tbs": round(achieved / 8000.0, 4)},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": args.steps * w.layers * 3,
+        "quantize": q_stats,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_oracle_decode_rate(w, layers)
+    return result
+
+
+def bench_quantize(args, dev, world):
+    w = W.PREFILL_64K_27L
+    n = w.total_tokens
+    hbm, bf16, src = peaks()
+    lays = []
+    for l in range(w.layers):
+        tau, gain = W.layer_constants(w, l)
+        pt = torch.as_tensor(W.page_table(w))
+        cache = R.PagedCache(int(pt.max()) + 1, pt, device=dev)
+        Rs = R.prepare_rotation(torch.as_tensor(W.rotation(w.seed + l)).to(dev))
+        c = W.latent_device(w, l, n, dev)
+        kr = W.rope_key_device(w, l, n, dev)
+        lays.append((cache, R.layer_params_init(tau, gain), Rs, c, kr))
+    req = torch.zeros(n, dtype=torch.int32, device=dev)
+    pos = torch.arange(n, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for cache, p, Rs, c, kr in lays:
+            R.quantize_append(cache, p, Rs, c, kr, req, pos)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world) / args.steps
+    tokens = n * w.layers
+    per_launch_ms = ms / w.layers
+    flops = 2.0 * n * 512 * 512                     # algorithmic (one bf16-exact GEMM)
+    bytes_ = n * (1024 + 128 + 288)
+    return {"workload": w.name, "tokens_per_s": round(tokens * world / (ms * 1e-3), 1),
+            "ms_per_step": round(ms, 4), "ms_per_launch": round(per_launch_ms, 4),
+            "roofline": {"bound": "tensor", "achieved": round(flops / (per_launch_ms * 1e-3) / 1e12, 1),
+                         "peak": bf16, "unit": "TFLOP/s",
+                         "frac": round(flops / (per_launch_ms * 1e-3) / 1e12 / bf16, 4),
+                         "executed_flops_factor": 2, "peak_source": src},
+            "hbm": {"achieved": round(bytes_ / (per_launch_ms * 1e-3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(bytes_ / (per_launch_ms * 1e-3) / 1e9 / hbm, 4)}}
+
+
+# ---------------------------------------------------------------- reference arm ----
+
+def run_reference(args, rank, world):
+    """The CPU oracle on this arm's workload: each step decodes one whole request of one
+    layer (262,144 tokens, fp64) on the host cores."""
+    from oracle import rolaq_oracle as O
+    w = W.DECODE_4x256K_27L
+    L = w.seq_lens[0]
+    rng = np.random.default_rng(w.seed)
+    tau, gain = W.layer_constants(w, 0)
+    packed = rng.integers(0, 256, size=(L, 128), dtype=np.uint8)
+    meta = np.stack([rng.standard_normal((L, 4)), np.abs(rng.standard_normal((L, 4))) + 0.5],
+                    axis=2).astype(np.float32)
+    kr = rng.standard_normal((L, 64))
+    qc = rng.standard_normal((w.heads, 512))
+    qr = rng.standard_normal((w.heads, 64))
+
+    def step():
+        O.decode_request(qc, qr, packed, meta, kr, tau, SM_SCALE)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = L * R.TOKEN_BYTES / dt / 1e9
+    return {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "impl": "reference",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seq_len": L, "heads": w.heads,
+                       "layers": w.layers},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": torch.get_num_threads(),
+                             "kind": "oracle",
+                             "sample": f"each step: one request x {L} tokens of one layer, fp64 oracle"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------------- plumbing -------
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 1)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    R.lib()
+    res = run_ours(args, rank, world, dev)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

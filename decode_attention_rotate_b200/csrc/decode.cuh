@@ -1,0 +1,505 @@
+// Absorbed-MLA decode attention over the packed 2-bit cache ("RoLaQ", §2.1, §3.3):
+// scores (q_c_rot . x + q_R . k_R) * sm_scale with x = mean + scale * level(code),
+// softmax over the request's tokens, 512-d latent readout in the rotated basis.
+//
+// Kernel A (rolaq_decode_split): one CTA per (work item, 16-head chunk).  A work item
+// is a run of whole pages of one request (split-K over the sequence).  The CTA holds
+// 9 warps:
+//   warp 8      producer: one 2-D bulk tensor copy per page (whole 18,432-byte page,
+//               128-byte swizzle) into an NSTAGE-deep ring of shared-memory stages;
+//   warps 0..7  two teams of four.  Team t owns tokens 32t..32t+31 of every page and
+//               keeps its own online-softmax state; inside a team, warp g owns
+//               content-channel group g (128 channels) and RoPE channels 16g..16g+15.
+// Per page and team: QK on the tensor cores (mma.sync m16n8k16, heads = M) with the
+// 2-bit codes turned into bf16 level fragments in registers (PRMT lookup), the group
+// metadata folded outside the MMA (q.x = mean * sum(q_g) + scale * (q_g . level)), a
+// cross-group reduction of the partial scores through shared memory, softmax, then
+// PV with the same level fragments transposed in registers (movmatrix) and the scale
+// folded into P (the mean term is a rank-1 update kept per head).
+// Kernel B (rolaq_decode_merge): log-sum-exp merge of the per-(item, team) partials.
+#pragma once
+#include "common.cuh"
+
+namespace rolaq {
+
+constexpr int kPageTok = ROLAQ_PAGE_TOKENS;
+constexpr int kPageBytes = ROLAQ_PAGE_BYTES;
+constexpr int kPageRows = ROLAQ_PAGE_BYTES / 128;   // 144 rows of 128 B
+constexpr int kNStage = 8;                          // half-page stages per team
+constexpr int kTStride = 40;                        // floats per head row of sT / sP
+constexpr int kDecodeThreads = 256;
+// A team stages its half of a page: 32 code rows, 8 metadata rows, 32 RoPE rows.
+constexpr int kHalfBytes = 9216;
+constexpr int kHalfMetaOff = 4096;                  // smem row 32
+constexpr int kHalfKrOff = 5120;                    // smem row 40
+
+struct DecodeArgs {
+    const int32_t* page_table;
+    int64_t num_pages;
+    int max_pages;
+    const __nv_bfloat16* prot;   // [batch][n_sink + n_recent][512] or null
+    int n_sink, n_recent;
+    const __nv_bfloat16* q;      // [batch][heads][512]
+    const __nv_bfloat16* qr;     // [batch][heads][64]
+    const int32_t* seq_lens;
+    int batch, heads;
+    float scale_log2;            // sm_scale * log2(e)
+    uint32_t lut_lo, lut_hi;     // low / high bytes of the four bf16 levels
+    int target_items;
+    float* ws_o;                 // [items][2][heads][512]
+    float2* ws_ml;               // [items][2][heads]  (running max (log2 units), sum)
+};
+
+struct DecodeSmem {
+    alignas(1024) uint8_t stage[2][kNStage][kHalfBytes];
+    float sT[2][4][16][kTStride];
+    float sP[2][16][kTStride];
+    float sAl[2][16];
+    alignas(8) uint64_t full[2][kNStage];
+    int valid[2][kNStage];
+    int plan[4];
+    int abort;
+};
+
+// ---- split plan --------------------------------------------------------------
+// pages_b = ceil(L_b / 64); chunk = max(1, ceil(sum_b pages_b / target)); request b
+// gets ceil(pages_b / chunk) items numbered consecutively in request order.  Executed
+// by one full warp; every lane returns the same values.
+struct PlanInfo { int b, first_page, n_pages, n_items, item_offset, chunk; };
+
+__device__ __forceinline__ int plan_chunk(const int32_t* seq_lens, int batch, int target) {
+    const int lane = threadIdx.x & 31;
+    long long total = 0;
+    for (int b = lane; b < batch; b += 32) {
+        int L = max(seq_lens[b], 0);
+        total += (L + kPageTok - 1) / kPageTok;
+    }
+    for (int o = 16; o; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
+    long long c = (total + target - 1) / target;
+    return (int)max(1LL, c);
+}
+
+// Locate work item `item` (or request `req` when item < 0).  n_items = total item count.
+__device__ PlanInfo plan_lookup(const int32_t* seq_lens, int batch, int target, int item,
+                                int req) {
+    const int lane = threadIdx.x & 31;
+    PlanInfo pi{-1, 0, 0, 0, 0, 0};
+    const int chunk = plan_chunk(seq_lens, batch, target);
+    pi.chunk = chunk;
+    int base = 0;
+    for (int b0 = 0; b0 < batch; b0 += 32) {
+        int b = b0 + lane;
+        int items = 0, pages = 0;
+        if (b < batch) {
+            pages = (max(seq_lens[b], 0) + kPageTok - 1) / kPageTok;
+            items = (pages + chunk - 1) / chunk;
+        }
+        int incl = items;
+        for (int o = 1; o < 32; o <<= 1) {
+            int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int excl = base + incl - items;
+        bool hit = (b < batch) && ((item >= 0) ? (item >= excl && item < excl + items) : (b == req));
+        unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (m) {
+            int src = __ffs(m) - 1;
+            int e = __shfl_sync(0xffffffffu, excl, src);
+            int it = __shfl_sync(0xffffffffu, items, src);
+            int pg = __shfl_sync(0xffffffffu, pages, src);
+            pi.b = b0 + src;
+            pi.item_offset = e;
+            pi.n_items = it;
+            if (item >= 0) {
+                int j = item - e;
+                pi.first_page = j * chunk;
+                pi.n_pages = min(chunk, pg - j * chunk);
+            } else {
+                pi.first_page = 0;
+                pi.n_pages = pg;
+            }
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (item >= 0 && pi.b < 0) pi.n_items = base;   // item past the end
+    return pi;
+}
+
+// Channel (within a 128-channel group) that QK k-slice s, MMA k index kk maps to.
+// Thread i = lane % 4 loads code bytes 8i..8i+7 of the group; its fragment values are
+// channels 32i + 16*(s/4) + 8*(kk/8) + 4*(kk%2) + s%4 (any channel order works for a
+// dot product as long as the query fragments follow it).
+__device__ __forceinline__ int qk_channel(int s, int kk) {
+    return 32 * ((kk & 7) >> 1) + 16 * (s >> 2) + 8 * (kk >> 3) + 4 * (kk & 1) + (s & 3);
+}
+
+// Four bf16 level pairs from one 32-bit word of codes (16 codes, 2 bit each).
+// Output r[k][0] = (level(code k), level(code 4+k)), r[k][1] = (code 8+k, code 12+k).
+// Selector byte for code c is c | (c + 4) << 4: PRMT takes the low level byte from
+// lut_lo[c] and the high byte from lut_hi[c].  (m >> 2k) * 0x11 spreads the code in each
+// byte to both nibbles; __umulhi(m, 0x11 << (16 - 2k)) does the same and moves bytes 2..3
+// down to 0..1 (every multiplier must fit in 32 bits).
+__device__ __forceinline__ void dequant_word(uint32_t w, uint32_t lo, uint32_t hi,
+                                             uint32_t (&r)[4][2]) {
+    uint32_t m0 = w & 0x03030303u;
+    r[0][0] = prmt(lo, hi, m0 * 0x11u + 0x40404040u);
+    r[0][1] = prmt(lo, hi, __umulhi(m0, 0x11u << 16) + 0x4040u);
+    uint32_t m1 = w & 0x0C0C0C0Cu;
+    r[1][0] = prmt(lo, hi, (m1 >> 2) * 0x11u + 0x40404040u);
+    r[1][1] = prmt(lo, hi, __umulhi(m1, 0x11u << 14) + 0x4040u);
+    uint32_t m2 = w & 0x30303030u;
+    r[2][0] = prmt(lo, hi, (m2 >> 4) * 0x11u + 0x40404040u);
+    r[2][1] = prmt(lo, hi, __umulhi(m2, 0x11u << 12) + 0x4040u);
+    uint32_t m3 = w & 0xC0C0C0C0u;
+    r[3][0] = prmt(lo, hi, __umulhi(m3, 0x11u << 26) + 0x40404040u);
+    r[3][1] = prmt(lo, hi, __umulhi(m3, 0x11u << 10) + 0x4040u);
+}
+
+// Issue the three copies of one team's half of page `k` (or mark it invalid).
+__device__ __forceinline__ void load_half_page(DecodeSmem& sm, const CUtensorMap* map32,
+                                               const CUtensorMap* map8, const DecodeArgs& args,
+                                               int team, int b, int page_idx, int k) {
+    const int st = k % kNStage;
+    long long pid = -1;
+    if (page_idx < args.max_pages) pid = args.page_table[(long long)b * args.max_pages + page_idx];
+    const uint32_t bar = smem_u32(&sm.full[team][st]);
+    if (pid >= 0 && pid < args.num_pages) {
+        sm.valid[team][st] = 1;
+        const int row0 = (int)(pid * kPageRows);
+        const uint32_t dst = smem_u32(sm.stage[team][st]);
+        mbar_arrive_expect_tx(bar, kHalfBytes);
+        tma_load_2d(dst, map32, 0, row0 + 32 * team, bar);
+        tma_load_2d(dst + kHalfMetaOff, map8, 0, row0 + 64 + 8 * team, bar);
+        tma_load_2d(dst + kHalfKrOff, map32, 0, row0 + 80 + 32 * team, bar);
+    } else {
+        sm.valid[team][st] = 0;
+        raise_status(ROLAQ_STATUS_BAD_PAGE);
+        mbar_arrive(bar);
+    }
+}
+
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+rolaq_decode_split(const __grid_constant__ CUtensorMap map32, const __grid_constant__ CUtensorMap map8,
+                   const DecodeArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hc = blockIdx.y;                 // 16-head chunk
+
+    if (warp == 0) {
+        PlanInfo pi = plan_lookup(args.seq_lens, args.batch, args.target_items,
+                                  (int)blockIdx.x, -1);
+        if (lane == 0) {
+            sm.plan[0] = pi.b;
+            sm.plan[1] = pi.first_page;
+            sm.plan[2] = pi.n_pages;
+        }
+    }
+    if (threadIdx.x == 32) {
+        for (int t = 0; t < 2; ++t)
+            for (int s = 0; s < kNStage; ++s) mbar_init(smem_u32(&sm.full[t][s]), 1);
+        sm.abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&map32);
+        prefetch_tmap(&map8);
+    }
+    __syncthreads();
+    const int b = sm.plan[0];
+    if (b < 0) return;                         // item past the end of the plan
+    const int first_page = sm.plan[1], n_pages = sm.plan[2];
+    const int L = args.seq_lens[b];
+    const int item = blockIdx.x;
+    const int team = warp >> 2, g = warp & 3;
+    const bool producer = (g == 0) && (lane == 0);
+    if (producer)
+        for (int k = 0; k < n_pages && k < kNStage; ++k)
+            load_half_page(sm, &map32, &map8, args, team, b, first_page + k, k);
+
+    // ---------------------------------------------------------------- consumers --
+    const int r = lane >> 2, i = lane & 3;     // mma fragment row group / thread in group
+    const int h0 = hc * 16;
+    const __nv_bfloat16* qrow0 = args.q + ((size_t)b * args.heads + h0 + r) * ROLAQ_D_C + 128 * g;
+    const __nv_bfloat16* qrow1 = qrow0 + 8 * ROLAQ_D_C;
+
+    // Query fragments for this warp's group, in the qk_channel order; row sums of q_g.
+    uint32_t qa[8][4];
+    float qs0 = 0.f, qs1 = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        const int c0 = qk_channel(s, 2 * i), c1 = qk_channel(s, 2 * i + 1);
+        const int c2 = qk_channel(s, 2 * i + 8), c3 = qk_channel(s, 2 * i + 9);
+        __nv_bfloat16 v00 = qrow0[c0], v01 = qrow0[c1], v02 = qrow0[c2], v03 = qrow0[c3];
+        __nv_bfloat16 v10 = qrow1[c0], v11 = qrow1[c1], v12 = qrow1[c2], v13 = qrow1[c3];
+        qa[s][0] = pack_bf16(__bfloat162float(v00), __bfloat162float(v01));
+        qa[s][1] = pack_bf16(__bfloat162float(v10), __bfloat162float(v11));
+        qa[s][2] = pack_bf16(__bfloat162float(v02), __bfloat162float(v03));
+        qa[s][3] = pack_bf16(__bfloat162float(v12), __bfloat162float(v13));
+        qs0 += __bfloat162float(v00) + __bfloat162float(v01) + __bfloat162float(v02) + __bfloat162float(v03);
+        qs1 += __bfloat162float(v10) + __bfloat162float(v11) + __bfloat162float(v12) + __bfloat162float(v13);
+    }
+    qs0 += __shfl_xor_sync(0xffffffffu, qs0, 1);
+    qs0 += __shfl_xor_sync(0xffffffffu, qs0, 2);
+    qs1 += __shfl_xor_sync(0xffffffffu, qs1, 1);
+    qs1 += __shfl_xor_sync(0xffffffffu, qs1, 2);
+    uint32_t qra[4];
+    {
+        const uint32_t* r0 = reinterpret_cast<const uint32_t*>(
+            args.qr + ((size_t)b * args.heads + h0 + r) * ROLAQ_D_R + 16 * g);
+        const uint32_t* r1 = r0 + 8 * ROLAQ_D_R / 2;
+        qra[0] = r0[i];
+        qra[1] = r1[i];
+        qra[2] = r0[4 + i];
+        qra[3] = r1[4 + i];
+    }
+
+    float o[8][2][4];
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) o[s][hf][c] = 0.f;
+    float u0 = 0.f, u1 = 0.f;                 // mean-term accumulators, rows r and r+8
+    float m_run = -INFINITY, l_run = 0.f;     // softmax state of head 4g + lane/8
+    const int hh = 4 * g + (lane >> 3), jj = lane & 7;
+
+    const uint32_t lut_lo = args.lut_lo, lut_hi = args.lut_hi;
+    const bool protect = args.n_sink > 0 || args.n_recent > 0;
+    const int recent_start = L - args.n_recent;
+
+    for (int k = 0; k < n_pages; ++k) {
+        const int st = k % kNStage;
+        // On a timeout the warp carries on with whatever the stage holds (the status
+        // word records it), so every warp still reaches the team barriers.
+        mbar_wait(smem_u32(&sm.full[team][st]), (k / kNStage) & 1, &sm.abort);
+        const int pos0 = (first_page + k) * kPageTok + 32 * team;
+        const int nvalid = sm.valid[team][st] ? min(max(L - pos0, 0), 32) : 0;
+        if (nvalid <= 0) {
+            // nothing of this half page is in the sequence; the barrier keeps every warp
+            // of the team past its wait before the stage is refilled
+            named_bar_sync(1 + team, 128);
+            if (producer && k + kNStage < n_pages)
+                load_half_page(sm, &map32, &map8, args, team, b, first_page + k + kNStage, k + kNStage);
+        } else {
+            const uint8_t* pg = sm.stage[team][st];
+            const bool mixed = protect && (pos0 < args.n_sink || pos0 + 32 > recent_start);
+
+            // ---- QK: dequantised level fragments for 4 n-tiles of 8 tokens -------
+            uint32_t bq[4][8][2];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const uint2 w = *reinterpret_cast<const uint2*>(pg + swz128(8 * nt + r, 32 * g + 8 * i));
+                uint32_t t[4][2];
+                dequant_word(w.x, lut_lo, lut_hi, t);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) { bq[nt][kk][0] = t[kk][0]; bq[nt][kk][1] = t[kk][1]; }
+                dequant_word(w.y, lut_lo, lut_hi, t);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) { bq[nt][4 + kk][0] = t[kk][0]; bq[nt][4 + kk][1] = t[kk][1]; }
+            }
+            if (mixed) {
+                // Protected tokens read their bf16 rotated content instead of the codes.
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    const int pos = pos0 + 8 * nt + r;
+                    if (pos < L && (pos < args.n_sink || pos >= recent_start)) {
+                        const int slot = pos < args.n_sink ? pos : args.n_sink + pos % args.n_recent;
+                        const uint4* src = reinterpret_cast<const uint4*>(
+                            args.prot + ((size_t)b * (args.n_sink + args.n_recent) + slot) * ROLAQ_D_C
+                            + 128 * g + 32 * i);
+                        uint32_t wv[16];
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4 v = src[q4];
+                            wv[4 * q4 + 0] = v.x; wv[4 * q4 + 1] = v.y;
+                            wv[4 * q4 + 2] = v.z; wv[4 * q4 + 3] = v.w;
+                        }
+#pragma unroll
+                        for (int s = 0; s < 8; ++s) {
+                            const int base = 16 * (s >> 2), kk = s & 3;
+                            const uint32_t sel = (kk & 1) ? 0x7632u : 0x5410u;
+                            bq[nt][s][0] = prmt(wv[(base + kk) >> 1], wv[(base + 4 + kk) >> 1], sel);
+                            bq[nt][s][1] = prmt(wv[(base + 8 + kk) >> 1], wv[(base + 12 + kk) >> 1], sel);
+                        }
+                    }
+                }
+            }
+
+            // metadata of the two tokens in each n-tile column pair: mean, scale
+            float mu[4][2], sc[4][2];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int t = 8 * nt + 2 * i + e;               // token row in the half
+                    const float2 ms = *reinterpret_cast<const float2*>(
+                        pg + swz128(32 + (t >> 2), (t & 3) * 32 + 8 * g));
+                    const int pos = pos0 + 8 * nt + 2 * i + e;
+                    const bool valid = (8 * nt + 2 * i + e) < nvalid;
+                    const bool prot = mixed && (pos < args.n_sink || pos >= recent_start);
+                    mu[nt][e] = (valid && !prot) ? ms.x : 0.f;
+                    sc[nt][e] = valid ? (prot ? 1.f : ms.y) : 0.f;
+                }
+
+            float acc[4][4];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
+#pragma unroll
+                for (int s = 0; s < 8; ++s) mma_bf16_16816(acc[nt], qa[s], bq[nt][s][0], bq[nt][s][1]);
+                // fold the group metadata: q.x = mean * sum(q_g) + scale * (q_g . level)
+                acc[nt][0] = fmaf(sc[nt][0], acc[nt][0], mu[nt][0] * qs0);
+                acc[nt][1] = fmaf(sc[nt][1], acc[nt][1], mu[nt][1] * qs0);
+                acc[nt][2] = fmaf(sc[nt][0], acc[nt][2], mu[nt][0] * qs1);
+                acc[nt][3] = fmaf(sc[nt][1], acc[nt][3], mu[nt][1] * qs1);
+                // RoPE part of the score for channels 16g..16g+15
+                const int row = 40 + 8 * nt + r;
+                const uint32_t kb0 = *reinterpret_cast<const uint32_t*>(pg + swz128(row, 32 * g + 4 * i));
+                const uint32_t kb1 = *reinterpret_cast<const uint32_t*>(pg + swz128(row, 32 * g + 16 + 4 * i));
+                mma_bf16_16816(acc[nt], qra, kb0, kb1);
+                const int tl = 8 * nt + 2 * i;
+                if (tl >= nvalid) { acc[nt][0] = -INFINITY; acc[nt][2] = -INFINITY; }
+                if (tl + 1 >= nvalid) { acc[nt][1] = -INFINITY; acc[nt][3] = -INFINITY; }
+                *reinterpret_cast<float2*>(&sm.sT[team][g][r][tl]) = make_float2(acc[nt][0], acc[nt][1]);
+                *reinterpret_cast<float2*>(&sm.sT[team][g][r + 8][tl]) = make_float2(acc[nt][2], acc[nt][3]);
+            }
+            named_bar_sync(1 + team, 128);
+            // every warp of the team is done reading this stage: refill it
+            if (producer && k + kNStage < n_pages)
+                load_half_page(sm, &map32, &map8, args, team, b, first_page + k + kNStage, k + kNStage);
+
+            // ---- softmax for heads 4g..4g+3 over this team's 32 tokens ------------
+            {
+                float sv[4];
+                float4 a0 = *reinterpret_cast<const float4*>(&sm.sT[team][0][hh][4 * jj]);
+                float4 a1 = *reinterpret_cast<const float4*>(&sm.sT[team][1][hh][4 * jj]);
+                float4 a2 = *reinterpret_cast<const float4*>(&sm.sT[team][2][hh][4 * jj]);
+                float4 a3 = *reinterpret_cast<const float4*>(&sm.sT[team][3][hh][4 * jj]);
+                sv[0] = (a0.x + a1.x + a2.x + a3.x) * args.scale_log2;
+                sv[1] = (a0.y + a1.y + a2.y + a3.y) * args.scale_log2;
+                sv[2] = (a0.z + a1.z + a2.z + a3.z) * args.scale_log2;
+                sv[3] = (a0.w + a1.w + a2.w + a3.w) * args.scale_log2;
+                float pm = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+                pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 1));
+                pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 2));
+                pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 4));
+                const float m_new = fmaxf(m_run, pm);
+                const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+                const float alpha = ex2(m_run - m_use);
+                float4 p;
+                p.x = ex2(sv[0] - m_use); p.y = ex2(sv[1] - m_use);
+                p.z = ex2(sv[2] - m_use); p.w = ex2(sv[3] - m_use);
+                float ps = (p.x + p.y) + (p.z + p.w);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+                ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+                l_run = l_run * alpha + ps;
+                m_run = m_new;
+                *reinterpret_cast<float4*>(&sm.sP[team][hh][4 * jj]) = p;
+                if (jj == 0) sm.sAl[team][hh] = alpha;
+            }
+            named_bar_sync(1 + team, 128);
+
+            // ---- PV: O_g[h, ch] += sum_t p * scale_t * level + (sum_t p * mean_t) -------
+            {
+                const float al0 = sm.sAl[team][r], al1 = sm.sAl[team][r + 8];
+                if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+                    for (int s = 0; s < 8; ++s)
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            o[s][hf][0] *= al0; o[s][hf][1] *= al0;
+                            o[s][hf][2] *= al1; o[s][hf][3] *= al1;
+                        }
+                }
+                u0 *= al0; u1 *= al1;
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    const int tl = 16 * ks + 2 * i;
+                    const float2 p00 = *reinterpret_cast<const float2*>(&sm.sP[team][r][tl]);
+                    const float2 p10 = *reinterpret_cast<const float2*>(&sm.sP[team][r + 8][tl]);
+                    const float2 p02 = *reinterpret_cast<const float2*>(&sm.sP[team][r][tl + 8]);
+                    const float2 p12 = *reinterpret_cast<const float2*>(&sm.sP[team][r + 8][tl + 8]);
+                    const int na = 2 * ks, nb = 2 * ks + 1;
+                    u0 += p00.x * mu[na][0] + p00.y * mu[na][1] + p02.x * mu[nb][0] + p02.y * mu[nb][1];
+                    u1 += p10.x * mu[na][0] + p10.y * mu[na][1] + p12.x * mu[nb][0] + p12.y * mu[nb][1];
+                    uint32_t pa[4];
+                    pa[0] = pack_bf16(p00.x * sc[na][0], p00.y * sc[na][1]);
+                    pa[1] = pack_bf16(p10.x * sc[na][0], p10.y * sc[na][1]);
+                    pa[2] = pack_bf16(p02.x * sc[nb][0], p02.y * sc[nb][1]);
+                    pa[3] = pack_bf16(p12.x * sc[nb][0], p12.y * sc[nb][1]);
+#pragma unroll
+                    for (int s = 0; s < 8; ++s)
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf)
+                            mma_bf16_16816(o[s][hf], pa, movmatrix_trans(bq[na][s][hf]),
+                                           movmatrix_trans(bq[nb][s][hf]));
+                }
+            }
+        }
+    }
+
+    // ---- write this team's partial: O + mean term, and (m, l) per head ---------
+    u0 += __shfl_xor_sync(0xffffffffu, u0, 1);
+    u0 += __shfl_xor_sync(0xffffffffu, u0, 2);
+    u1 += __shfl_xor_sync(0xffffffffu, u1, 1);
+    u1 += __shfl_xor_sync(0xffffffffu, u1, 2);
+    const size_t part = (size_t)item * 2 + team;
+    float* out0 = args.ws_o + (part * args.heads + h0 + r) * ROLAQ_D_C + 128 * g;
+    float* out1 = out0 + 8 * ROLAQ_D_C;
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const int ch = 32 * i + 16 * (s >> 2) + 8 * hf + 4 * e + (s & 3);
+                out0[ch] = o[s][hf][e] + u0;
+                out1[ch] = o[s][hf][2 + e] + u1;
+            }
+    if (jj == 0) args.ws_ml[part * args.heads + h0 + hh] = make_float2(m_run, l_run);
+}
+
+// ---- merge --------------------------------------------------------------------
+// grid (batch, heads), 128 threads: out[b,h,:] = sum_i w_i o_i / sum_i w_i l_i with
+// w_i = 2^(m_i - max m); lse = (max m + log2(sum w l)) * ln 2.
+__global__ void __launch_bounds__(128)
+rolaq_decode_merge(const float* __restrict__ ws_o, const float2* __restrict__ ws_ml,
+                   const int32_t* seq_lens, int batch, int heads, int target,
+                   float* __restrict__ out, float* __restrict__ lse) {
+    __shared__ int s_plan[2];
+    const int b = blockIdx.x, h = blockIdx.y;
+    if (threadIdx.x < 32) {
+        PlanInfo pi = plan_lookup(seq_lens, batch, target, -1, b);
+        if (threadIdx.x == 0) { s_plan[0] = pi.item_offset; s_plan[1] = pi.n_items; }
+    }
+    __syncthreads();
+    const int p0 = 2 * s_plan[0], np = 2 * s_plan[1];
+    float M = -INFINITY;
+    for (int p = 0; p < np; ++p) M = fmaxf(M, ws_ml[(size_t)(p0 + p) * heads + h].x);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.f;
+    if (M != -INFINITY) {
+        for (int p = 0; p < np; ++p) {
+            const float2 ml = ws_ml[(size_t)(p0 + p) * heads + h];
+            if (ml.y == 0.f) continue;
+            const float w = exp2f(ml.x - M);
+            den += w * ml.y;
+            const float4 v = reinterpret_cast<const float4*>(
+                ws_o + ((size_t)(p0 + p) * heads + h) * ROLAQ_D_C)[threadIdx.x];
+            acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+        }
+    }
+    float4 res = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (den > 0.f) {
+        const float inv = 1.f / den;
+        res = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+    reinterpret_cast<float4*>(out + ((size_t)b * heads + h) * ROLAQ_D_C)[threadIdx.x] = res;
+    if (lse && threadIdx.x == 0)
+        lse[(size_t)b * heads + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+}
+
+}  // namespace rolaq

@@ -1,0 +1,317 @@
+// Write path ("RoLaQ", §3.2, §3.3, §A.3): y = c . R on the 5th-generation tensor cores,
+// then per 128-coordinate group: mean, population std, four-level codes by tau, 2-bit
+// packing, (mean, gain*std) metadata, the bf16 RoPE key copy and, for protected tokens,
+// bf16(y) into the side store.
+//
+// rolaq_quantize_kernel is persistent (one CTA per SM).  A tile is 128 tokens; it is
+// produced as two halves of 256 output coordinates (two groups each).  Warp roles:
+//   warp 8   producer: bulk tensor copies of c (128 x 32) and of both R planes
+//            (256 x 32 each) per 32-wide K step into a 4-deep shared-memory ring;
+//   warp 9   allocates 512 TMEM columns and issues tcgen05.mma (M=128, N=256, K=16,
+//            bf16 in, fp32 accumulate) for R_hi and R_lo into one accumulator, so
+//            y = c.R_hi + c.R_lo carries ~2^-17 relative error; the two halves use
+//            separate accumulators (TMEM columns 0..255 / 256..511), so the epilogue
+//            of one half overlaps the MMAs of the next;
+//   warps 0..7  epilogue: warp e reads TMEM lanes 32*(e%4).. (one token per thread) and
+//            quantizes group 2*half + e/4 of that token.
+#pragma once
+#include "common.cuh"
+
+namespace rolaq {
+
+constexpr int kQTileM = 128;
+constexpr int kQHalfN = 256;
+constexpr int kQK = 32;                       // K per stage (64-byte rows, 64B swizzle)
+constexpr int kQStages = 4;
+constexpr int kQKSteps = ROLAQ_D_C / kQK;     // 16
+constexpr int kQThreads = 320;
+constexpr uint32_t kQStageABytes = kQTileM * kQK * 2;     // 8 KB
+constexpr uint32_t kQStageBBytes = kQHalfN * kQK * 2;     // 16 KB per plane
+constexpr uint32_t kQStageTx = kQStageABytes + 2 * kQStageBBytes;
+
+struct QuantArgs {
+    uint8_t* pages;
+    int64_t num_pages;
+    const int32_t* page_table;
+    int max_pages, batch;
+    __nv_bfloat16* prot;
+    int n_sink, n_recent;
+    const int32_t* req;
+    const int32_t* pos;
+    const int32_t* seq_lens;
+    const __nv_bfloat16* k_r;   // [n][64]
+    int n;
+    float tau, gain;
+};
+
+struct QuantSmem {
+    alignas(1024) uint8_t a[kQStages][kQStageABytes];
+    alignas(1024) uint8_t bh[kQStages][kQStageBBytes];
+    alignas(1024) uint8_t bl[kQStages][kQStageBBytes];
+    alignas(8) uint64_t full[kQStages];
+    uint64_t empty[kQStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Shared-memory matrix descriptor: K-major operand, 64-byte rows with 64B swizzle,
+// 8-row core groups 512 bytes apart.
+__device__ __forceinline__ uint64_t umma_desc_sw64(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (32ull << 32) | (1ull << 46) |
+           (4ull << 61);
+}
+// Instruction descriptor: bf16 x bf16 -> f32, both K-major, M = 128, N = 256.
+constexpr uint32_t kQIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kQHalfN >> 3) << 17) |
+                             ((uint32_t)(kQTileM >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(tmem_d), "l"(da), "l"(db), "r"(kQIdesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// 32 lanes x 32 columns of fp32 from TMEM, one row (lane) per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t* u = reinterpret_cast<uint32_t*>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+          "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]),
+          "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]),
+          "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]), "=r"(u[25]),
+          "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Quantize one 128-coordinate group of one token straight from TMEM (this thread's
+// lane, columns col..col+127), streaming 32 columns at a time in three passes: mean,
+// population std, then codes (and the bf16 copy for a protected token).  All lanes of
+// the warp must call it (the TMEM loads are warp-wide); `store` is false for lanes
+// without a valid target.
+__device__ __forceinline__ void quantize_group_tmem(uint32_t col, float tau, float gain, bool store,
+                                                    uint8_t* dst_codes, float* dst_meta,
+                                                    __nv_bfloat16* dst_prot) {
+    float t[32];
+    float s = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        tmem_ld32(col + 32 * c, t);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) s += t[j];
+    }
+    const float mean = s * (1.f / 128.f);
+    float ss = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+        tmem_ld32(col + 32 * c, t);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float d = t[j] - mean;
+            ss = fmaf(d, d, ss);
+        }
+    }
+    const float sd = sqrtf(ss * (1.f / 128.f));
+    // z = (y - mean) / sd against -tau, 0, tau; a group with sd == 0 gets z = 0.
+    const float inv = sd > 0.f ? 1.f / sd : 0.f;
+    uint32_t w[8];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        tmem_ld32(col + 32 * c, t);
+        tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t acc = 0;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float z = (t[16 * h + j] - mean) * inv;
+                const uint32_t code = (uint32_t)(z >= -tau) + (uint32_t)(z >= 0.f) + (uint32_t)(z >= tau);
+                acc |= code << (2 * j);
+            }
+            w[2 * c + h] = acc;
+        }
+        if (store && dst_prot) {
+            uint4* dp = reinterpret_cast<uint4*>(dst_prot + 32 * c);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8)
+                dp[q8] = make_uint4(pack_bf16(t[8 * q8 + 0], t[8 * q8 + 1]), pack_bf16(t[8 * q8 + 2], t[8 * q8 + 3]),
+                                    pack_bf16(t[8 * q8 + 4], t[8 * q8 + 5]), pack_bf16(t[8 * q8 + 6], t[8 * q8 + 7]));
+        }
+    }
+    if (store) {
+        uint4* dc = reinterpret_cast<uint4*>(dst_codes);
+        dc[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dc[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        *reinterpret_cast<float2*>(dst_meta) = make_float2(mean, gain * sd);
+    }
+}
+
+__global__ void __launch_bounds__(kQThreads, 1)
+rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
+                      const __grid_constant__ CUtensorMap map_r, const QuantArgs args) {
+    extern __shared__ uint8_t smem_raw[];
+    QuantSmem& sm = *reinterpret_cast<QuantSmem*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = (args.n + kQTileM - 1) / kQTileM;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kQStages; ++s) {
+            mbar_init(smem_u32(&sm.full[s]), 1);
+            mbar_init(smem_u32(&sm.empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&sm.tfull[a]), 1);
+            mbar_init(smem_u32(&sm.tempty[a]), 8);
+        }
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 9) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
+                     :: "r"(smem_u32(&sm.tmem_base)) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (warp == 8 && lane == 0) { prefetch_tmap(&map_c); prefetch_tmap(&map_r); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 8) {
+        // ------------------------------------------------------------- producer --
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x)
+                for (int nh = 0; nh < 2 && ok; ++nh)
+                    for (int kc = 0; kc < kQKSteps; ++kc, ++it) {
+                        const int st = it % kQStages;
+                        if (it >= kQStages && !mbar_wait(smem_u32(&sm.empty[st]), ((it / kQStages) - 1) & 1, &sm.abort)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t fb = smem_u32(&sm.full[st]);
+                        mbar_arrive_expect_tx(fb, kQStageTx);
+                        tma_load_2d(smem_u32(sm.a[st]), &map_c, kc * kQK, tile * kQTileM, fb);
+                        tma_load_2d(smem_u32(sm.bh[st]), &map_r, kc * kQK, nh * kQHalfN, fb);
+                        tma_load_2d(smem_u32(sm.bl[st]), &map_r, kc * kQK, ROLAQ_D_C + nh * kQHalfN, fb);
+                    }
+        }
+    } else if (warp == 9) {
+        // ----------------------------------------------------------------- MMA ----
+        if (lane == 0) {
+            uint32_t it = 0, job = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x)
+                for (int nh = 0; nh < 2 && ok; ++nh, ++job) {
+                    const uint32_t use = job >> 1;
+                    if (use >= 1 && !mbar_wait(smem_u32(&sm.tempty[nh]), (use - 1) & 1, &sm.abort)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d = tmem + (uint32_t)(nh * kQHalfN);
+                    for (int kc = 0; kc < kQKSteps; ++kc, ++it) {
+                        const int st = it % kQStages;
+                        if (!mbar_wait(smem_u32(&sm.full[st]), (it / kQStages) & 1, &sm.abort)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t sa = smem_u32(sm.a[st]);
+                        const uint32_t sbh = smem_u32(sm.bh[st]), sbl = smem_u32(sm.bl[st]);
+#pragma unroll
+                        for (int k16 = 0; k16 < 2; ++k16) {
+                            const uint64_t da = umma_desc_sw64(sa + 32 * k16);
+                            umma_bf16(d, da, umma_desc_sw64(sbh + 32 * k16), (kc | k16) != 0);
+                            umma_bf16(d, da, umma_desc_sw64(sbl + 32 * k16), 1u);
+                        }
+                        umma_commit(smem_u32(&sm.empty[st]));
+                    }
+                    if (ok) umma_commit(smem_u32(&sm.tfull[nh]));
+                }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue ----
+        const int q = warp & 3, gg = warp >> 2;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        uint32_t job = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x)
+            for (int nh = 0; nh < 2; ++nh, ++job) {
+                const bool got = mbar_wait(smem_u32(&sm.tfull[nh]), (job >> 1) & 1, &sm.abort);
+                tc_fence_after();
+                const int tok = tile * kQTileM + 32 * q + lane;
+                const int g = 2 * nh + gg;
+                long long pid = -1;
+                int rq = -1, ps = 0;
+                if (got && tok < args.n) {
+                    rq = args.req[tok];
+                    ps = args.pos[tok];
+                    if (rq >= 0 && rq < args.batch && ps >= 0 && (ps / ROLAQ_PAGE_TOKENS) < args.max_pages) {
+                        pid = args.page_table[(long long)rq * args.max_pages + ps / ROLAQ_PAGE_TOKENS];
+                        if (pid >= args.num_pages) pid = -1;
+                    }
+                    if (pid < 0 && nh == 0 && gg == 0) raise_status(ROLAQ_STATUS_BAD_SLOT);
+                }
+                const bool store = pid >= 0;
+                uint8_t* page = args.pages + (store ? pid : 0) * (long long)ROLAQ_PAGE_BYTES;
+                const int row = ps % ROLAQ_PAGE_TOKENS;
+                __nv_bfloat16* prot = nullptr;
+                if (store && args.prot) {
+                    const int nslot = args.n_sink + args.n_recent;
+                    if (ps < args.n_sink)
+                        prot = args.prot + ((size_t)rq * nslot + ps) * ROLAQ_D_C + 128 * g;
+                    else if (args.n_recent > 0 && ps >= args.seq_lens[rq] - args.n_recent)
+                        prot = args.prot + ((size_t)rq * nslot + args.n_sink + ps % args.n_recent) * ROLAQ_D_C + 128 * g;
+                }
+                quantize_group_tmem(tmem + lane_base + (uint32_t)(nh * kQHalfN + gg * 128), args.tau, args.gain,
+                                    store, page + ROLAQ_PAGE_CODES_OFFSET + row * ROLAQ_CODE_BYTES + 32 * g,
+                                    reinterpret_cast<float*>(page + ROLAQ_PAGE_META_OFFSET + row * ROLAQ_META_BYTES) + 2 * g,
+                                    prot);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[nh]));
+                if (store && nh == 0 && gg == 0) {
+                    const uint4* src = reinterpret_cast<const uint4*>(args.k_r + (size_t)tok * ROLAQ_D_R);
+                    uint4* dst = reinterpret_cast<uint4*>(page + ROLAQ_PAGE_KR_OFFSET + row * ROLAQ_KR_BYTES);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) dst[j] = src[j];
+                }
+            }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" :: "r"(tmem) : "memory");
+    }
+}
+
+// R (fp32 [512 in][512 out], y = c . R) -> two bf16 planes [2][512 out][512 in]: the
+// nearest bf16 of R^T and the nearest bf16 of the remainder.
+__global__ void rolaq_split_rotation(const float* __restrict__ R, __nv_bfloat16* __restrict__ out) {
+    const int o = blockIdx.x;                  // output coordinate (row of R^T)
+    for (int k = threadIdx.x; k < ROLAQ_D_C; k += blockDim.x) {
+        const float x = R[(size_t)k * ROLAQ_D_C + o];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+        out[(size_t)o * ROLAQ_D_C + k] = hi;
+        out[(size_t)ROLAQ_D_C * ROLAQ_D_C + (size_t)o * ROLAQ_D_C + k] = lo;
+    }
+}
+
+}  // namespace rolaq

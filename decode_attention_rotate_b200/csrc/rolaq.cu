@@ -1,0 +1,286 @@
+// librolaq: C ABI over the sm_100a kernels of the 2-bit rotated MLA cache.
+// One translation unit so the device status word is a single symbol.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+#include <mutex>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "quantize.cuh"
+
+using namespace rolaq;
+
+namespace {
+
+constexpr int kVersion = 100;   // 0.1.0
+constexpr int kMaxDevices = 64;
+
+int device_sms(int dev) {
+    static int cache[kMaxDevices] = {0};
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+int current_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    return device_sms(dev);
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, void* base, uint64_t inner, uint64_t rows,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// bf16 bit pattern of an fp32 value, round to nearest even (finite inputs).
+uint16_t bf16_bits(float x) {
+    uint32_t u;
+    memcpy(&u, &x, 4);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+int check_cache(const rolaq_cache* c) {
+    if (!c || !c->pages_dev || !c->page_table_dev || c->num_pages <= 0 || c->batch <= 0 ||
+        c->max_pages_per_seq <= 0)
+        return ROLAQ_EINVAL;
+    if (!aligned(c->pages_dev, 256) || !aligned(c->page_table_dev, 4)) return ROLAQ_EINVAL;
+    if (c->n_sink < 0 || c->n_recent < 0) return ROLAQ_EINVAL;
+    if ((c->n_sink > 0 || c->n_recent > 0) && (!c->prot_dev || !aligned(c->prot_dev, 16)))
+        return ROLAQ_EINVAL;
+    if (c->num_pages * (int64_t)(ROLAQ_PAGE_BYTES / 128) >= (int64_t)INT32_MAX) return ROLAQ_EINVAL;
+    return ROLAQ_OK;
+}
+
+int check_params(const rolaq_layer_params* p) {
+    if (!p || !(p->tau > 0.f) || !(p->gain > 0.f) || !isfinite(p->tau) || !isfinite(p->gain) ||
+        !(p->level_a > 0.f) || !(p->level_b > p->level_a))
+        return ROLAQ_EINVAL;
+    return ROLAQ_OK;
+}
+
+int decode_target_items(int heads) {
+    const int chunks = heads / 16;
+    return (current_sms() + chunks - 1) / chunks;
+}
+
+size_t decode_ws_bytes(int batch, int heads) {
+    const size_t items = (size_t)decode_target_items(heads) + (size_t)batch;
+    const size_t o = items * 2 * heads * ROLAQ_D_C * sizeof(float);
+    const size_t ml = items * 2 * heads * sizeof(float2);
+    return o + ml;
+}
+
+int launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ROLAQ_OK : ROLAQ_ECUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rolaq_version(void) { return kVersion; }
+
+const char* rolaq_strerror(int code) {
+    switch (code) {
+        case ROLAQ_OK: return "ok";
+        case ROLAQ_EINVAL: return "invalid argument (null or misaligned pointer, bad size or shape)";
+        case ROLAQ_ENOSPACE: return "workspace too small";
+        case ROLAQ_ECUDA: return "CUDA call failed";
+        case ROLAQ_EUNSUPPORTED: return "unsupported shape";
+        default: return "unknown error";
+    }
+}
+
+int rolaq_layer_params_init(rolaq_layer_params* p, float tau, float gain) {
+    if (!p || !isfinite(tau) || !isfinite(gain) || !(tau > 0.f) || !(gain > 0.f)) return ROLAQ_EINVAL;
+    const double t = tau;
+    const double inv_sqrt_2pi = 0.39894228040143267794;
+    const double phi0 = inv_sqrt_2pi, phit = inv_sqrt_2pi * exp(-0.5 * t * t);
+    const double Phit = 0.5 * (1.0 + erf(t / sqrt(2.0)));
+    const double a = (phi0 - phit) / (Phit - 0.5);
+    const double b = phit / (0.5 * erfc(t / sqrt(2.0)));
+    p->tau = tau;
+    p->gain = gain;
+    p->level_a = (float)a;
+    p->level_b = (float)b;
+    return ROLAQ_OK;
+}
+
+int rolaq_prepare_rotation(const float* R_dev, void* R_split_dev, void* stream) {
+    if (!R_dev || !R_split_dev || !aligned(R_dev, 4) || !aligned(R_split_dev, 16)) return ROLAQ_EINVAL;
+    rolaq_split_rotation<<<ROLAQ_D_C, 128, 0, (cudaStream_t)stream>>>(
+        R_dev, reinterpret_cast<__nv_bfloat16*>(R_split_dev));
+    return launch_status();
+}
+
+int rolaq_quantize_append(const rolaq_cache* cache, const rolaq_layer_params* p,
+                          const void* R_split_dev, const void* c_dev, const void* k_R_dev,
+                          const int32_t* req_dev, const int32_t* pos_dev,
+                          const int32_t* seq_lens_dev, int n, void* stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if ((rc = check_params(p))) return rc;
+    if (n < 0) return ROLAQ_EINVAL;
+    if (n == 0) return ROLAQ_OK;
+    if (!R_split_dev || !c_dev || !k_R_dev || !req_dev || !pos_dev) return ROLAQ_EINVAL;
+    if (!aligned(R_split_dev, 16) || !aligned(c_dev, 16) || !aligned(k_R_dev, 16) ||
+        !aligned(req_dev, 4) || !aligned(pos_dev, 4))
+        return ROLAQ_EINVAL;
+    if (cache->n_recent > 0 && !seq_lens_dev) return ROLAQ_EINVAL;
+
+    CUtensorMap map_c, map_r;
+    if (!encode_2d(&map_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(c_dev), ROLAQ_D_C,
+                   (uint64_t)n, ROLAQ_D_C * 2, kQK, kQTileM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_2d(&map_r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(R_split_dev), ROLAQ_D_C,
+                   2 * ROLAQ_D_C, ROLAQ_D_C * 2, kQK, kQHalfN, CU_TENSOR_MAP_SWIZZLE_64B))
+        return ROLAQ_ECUDA;
+
+    QuantArgs a;
+    a.pages = reinterpret_cast<uint8_t*>(cache->pages_dev);
+    a.num_pages = cache->num_pages;
+    a.page_table = cache->page_table_dev;
+    a.max_pages = cache->max_pages_per_seq;
+    a.batch = cache->batch;
+    a.prot = (cache->n_sink + cache->n_recent > 0) ? reinterpret_cast<__nv_bfloat16*>(cache->prot_dev) : nullptr;
+    a.n_sink = cache->n_sink;
+    a.n_recent = cache->n_recent;
+    a.req = req_dev;
+    a.pos = pos_dev;
+    a.seq_lens = seq_lens_dev;
+    a.k_r = reinterpret_cast<const __nv_bfloat16*>(k_R_dev);
+    a.n = n;
+    a.tau = p->tau;
+    a.gain = p->gain;
+
+    const size_t smem = sizeof(QuantSmem) + 1024;
+    static std::once_flag attr_once;
+    std::call_once(attr_once, [smem] {
+        cudaFuncSetAttribute(rolaq_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
+    const int tiles = (n + kQTileM - 1) / kQTileM;
+    const int grid = tiles < current_sms() ? tiles : current_sms();
+    rolaq_quantize_kernel<<<grid, kQThreads, smem, (cudaStream_t)stream>>>(map_c, map_r, a);
+    return launch_status();
+}
+
+size_t rolaq_decode_workspace_bytes(int batch, int heads) {
+    if (batch <= 0 || heads <= 0 || heads % 16) return 0;
+    return decode_ws_bytes(batch, heads);
+}
+
+int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
+                      const void* q_c_rot_dev, const void* q_R_dev,
+                      const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
+                      float* out_dev, float* lse_dev,
+                      void* workspace_dev, size_t workspace_bytes, void* stream) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if ((rc = check_params(p))) return rc;
+    if (heads <= 0 || heads % 16) return ROLAQ_EUNSUPPORTED;
+    if (batch <= 0 || batch > cache->batch) return ROLAQ_EINVAL;
+    if (!q_c_rot_dev || !q_R_dev || !seq_lens_dev || !out_dev || !workspace_dev) return ROLAQ_EINVAL;
+    if (!aligned(q_c_rot_dev, 4) || !aligned(q_R_dev, 4) || !aligned(seq_lens_dev, 4) ||
+        !aligned(out_dev, 16) || !aligned(workspace_dev, 16) || (lse_dev && !aligned(lse_dev, 4)))
+        return ROLAQ_EINVAL;
+    if (!isfinite(sm_scale)) return ROLAQ_EINVAL;
+    if (workspace_bytes < decode_ws_bytes(batch, heads)) return ROLAQ_ENOSPACE;
+
+    // The pool as rows of 128 B; boxes of 32 rows (codes, k_R) and 8 rows (metadata).
+    CUtensorMap map32, map8;
+    const uint64_t rows = (uint64_t)cache->num_pages * (ROLAQ_PAGE_BYTES / 128);
+    if (!encode_2d(&map32, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache->pages_dev, 128, rows, 128, 128, 32,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&map8, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache->pages_dev, 128, rows, 128, 128, 8,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return ROLAQ_ECUDA;
+
+    const int target = decode_target_items(heads);
+    const int items_cap = target + batch;
+    DecodeArgs a;
+    a.page_table = cache->page_table_dev;
+    a.num_pages = cache->num_pages;
+    a.max_pages = cache->max_pages_per_seq;
+    a.prot = reinterpret_cast<const __nv_bfloat16*>(cache->prot_dev);
+    a.n_sink = cache->n_sink;
+    a.n_recent = cache->n_recent;
+    a.q = reinterpret_cast<const __nv_bfloat16*>(q_c_rot_dev);
+    a.qr = reinterpret_cast<const __nv_bfloat16*>(q_R_dev);
+    a.seq_lens = seq_lens_dev;
+    a.batch = batch;
+    a.heads = heads;
+    a.scale_log2 = sm_scale * 1.4426950408889634f;
+    const float lv[4] = {-p->level_b, -p->level_a, p->level_a, p->level_b};
+    uint32_t lo = 0, hi = 0;
+    for (int c = 0; c < 4; ++c) {
+        const uint16_t bits = bf16_bits(lv[c]);
+        lo |= (uint32_t)(bits & 0xFFu) << (8 * c);
+        hi |= (uint32_t)(bits >> 8) << (8 * c);
+    }
+    a.lut_lo = lo;
+    a.lut_hi = hi;
+    a.target_items = target;
+    a.ws_o = reinterpret_cast<float*>(workspace_dev);
+    a.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace_dev) +
+                                        (size_t)items_cap * 2 * heads * ROLAQ_D_C * sizeof(float));
+
+    const size_t smem = sizeof(DecodeSmem) + 1024;
+    static std::once_flag attr_once;
+    std::call_once(attr_once, [smem] {
+        cudaFuncSetAttribute(rolaq_decode_split, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
+    cudaStream_t s = (cudaStream_t)stream;
+    rolaq_decode_split<<<dim3(items_cap, heads / 16), kDecodeThreads, smem, s>>>(map32, map8, a);
+    if ((rc = launch_status())) return rc;
+    rolaq_decode_merge<<<dim3(batch, heads), 128, 0, s>>>(a.ws_o, a.ws_ml, seq_lens_dev, batch, heads,
+                                                         target, out_dev, lse_dev);
+    return launch_status();
+}
+
+int rolaq_get_status(int* bits, void* stream) {
+    if (!bits) return ROLAQ_EINVAL;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return ROLAQ_ECUDA;
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return ROLAQ_ECUDA;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return ROLAQ_ECUDA;
+    *bits = (int)v;
+    return ROLAQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,216 @@
+"""Python binding of librolaq (argument marshalling only).
+
+Every function forwards to the C entry point of the same name in librolaq.so; all
+computation happens in the library's CUDA kernels.  Tensors are torch CUDA tensors
+(PyTorch provides device memory and streams here).  There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+D_C = 512
+D_R = 64
+PAGE_TOKENS = 64
+PAGE_BYTES = 18432
+TOKEN_BYTES = 288
+RSPLIT_BYTES = 2 * 512 * 512 * 2
+
+STATUS_BAD_PAGE = 1
+STATUS_BAD_SLOT = 2
+STATUS_TIMEOUT = 4
+
+
+class RolaqError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed: {code} ({strerror(code)})")
+        self.code = code
+
+
+class rolaq_cache(ctypes.Structure):
+    _fields_ = [
+        ("pages_dev", ctypes.c_void_p),
+        ("num_pages", ctypes.c_int64),
+        ("page_table_dev", ctypes.c_void_p),
+        ("batch", ctypes.c_int32),
+        ("max_pages_per_seq", ctypes.c_int32),
+        ("prot_dev", ctypes.c_void_p),
+        ("n_sink", ctypes.c_int32),
+        ("n_recent", ctypes.c_int32),
+    ]
+
+
+class rolaq_layer_params(ctypes.Structure):
+    _fields_ = [
+        ("tau", ctypes.c_float),
+        ("gain", ctypes.c_float),
+        ("level_a", ctypes.c_float),
+        ("level_b", ctypes.c_float),
+    ]
+
+
+_LIB = None
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"librolaq.so not built ({path}); run decode_attention_rotate_b200.build")
+        L = ctypes.CDLL(path)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        P = ctypes.POINTER
+        L.rolaq_version.restype = i32
+        L.rolaq_strerror.restype = ctypes.c_char_p
+        L.rolaq_strerror.argtypes = [i32]
+        L.rolaq_layer_params_init.restype = i32
+        L.rolaq_layer_params_init.argtypes = [P(rolaq_layer_params), ctypes.c_float, ctypes.c_float]
+        L.rolaq_prepare_rotation.restype = i32
+        L.rolaq_prepare_rotation.argtypes = [vp, vp, vp]
+        L.rolaq_quantize_append.restype = i32
+        L.rolaq_quantize_append.argtypes = [P(rolaq_cache), P(rolaq_layer_params), vp, vp, vp, vp, vp,
+                                            vp, i32, vp]
+        L.rolaq_decode_workspace_bytes.restype = sz
+        L.rolaq_decode_workspace_bytes.argtypes = [i32, i32]
+        L.rolaq_decode_attn.restype = i32
+        L.rolaq_decode_attn.argtypes = [P(rolaq_cache), P(rolaq_layer_params), vp, vp, vp, i32, i32,
+                                        ctypes.c_float, vp, vp, vp, sz, vp]
+        L.rolaq_get_status.restype = i32
+        L.rolaq_get_status.argtypes = [P(ctypes.c_int), vp]
+        _LIB = L
+    return _LIB
+
+
+def header_functions() -> list:
+    """Names of the functions include/rolaq.h declares."""
+    hdr = os.path.join(_build.INCLUDE, "rolaq.h")
+    text = open(hdr).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rolaq_[a-z_0-9]+)\s*\(", text)))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != 0:
+        raise RolaqError(fn, rc)
+
+
+def version() -> int:
+    return lib().rolaq_version()
+
+
+def strerror(code: int) -> str:
+    return lib().rolaq_strerror(code).decode()
+
+
+def layer_params_init(tau: float, gain: float) -> rolaq_layer_params:
+    p = rolaq_layer_params()
+    _check("rolaq_layer_params_init", lib().rolaq_layer_params_init(ctypes.byref(p), tau, gain))
+    return p
+
+
+def prepare_rotation(R: torch.Tensor, R_split: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """R: fp32 [512, 512] CUDA (y = c @ R).  Returns the bf16 operand [2, 512, 512]."""
+    assert R.dtype == torch.float32 and tuple(R.shape) == (D_C, D_C)
+    if R_split is None:
+        R_split = torch.empty((2, D_C, D_C), dtype=torch.bfloat16, device=R.device)
+    _check("rolaq_prepare_rotation", lib().rolaq_prepare_rotation(_ptr(R), _ptr(R_split), _stream(stream)))
+    return R_split
+
+
+class PagedCache:
+    """Device buffers of one layer's cache plus the C descriptor that points at them."""
+
+    def __init__(self, num_pages: int, page_table: torch.Tensor, n_sink: int = 0, n_recent: int = 0,
+                 device="cuda", pages: Optional[torch.Tensor] = None):
+        self.page_table = page_table.to(device=device, dtype=torch.int32).contiguous()
+        self.batch, self.max_pages = self.page_table.shape
+        self.num_pages = int(num_pages)
+        self.pages = pages if pages is not None else torch.zeros(
+            self.num_pages * PAGE_BYTES, dtype=torch.uint8, device=device)
+        self.n_sink, self.n_recent = int(n_sink), int(n_recent)
+        nslot = self.n_sink + self.n_recent
+        self.prot = (torch.zeros((self.batch, nslot, D_C), dtype=torch.bfloat16, device=device)
+                     if nslot else None)
+
+    def desc(self) -> rolaq_cache:
+        c = rolaq_cache()
+        c.pages_dev = _ptr(self.pages)
+        c.num_pages = self.num_pages
+        c.page_table_dev = _ptr(self.page_table)
+        c.batch = self.batch
+        c.max_pages_per_seq = self.max_pages
+        c.prot_dev = _ptr(self.prot) if self.prot is not None else None
+        c.n_sink = self.n_sink
+        c.n_recent = self.n_recent
+        return c
+
+
+def quantize_append(cache: PagedCache, params: rolaq_layer_params, R_split: torch.Tensor,
+                    c: torch.Tensor, k_r: torch.Tensor, req: torch.Tensor, pos: torch.Tensor,
+                    seq_lens: Optional[torch.Tensor] = None, stream=None) -> None:
+    n = int(c.shape[0])
+    assert c.dtype == torch.bfloat16 and k_r.dtype == torch.bfloat16
+    assert req.dtype == torch.int32 and pos.dtype == torch.int32
+    d = cache.desc()
+    _check("rolaq_quantize_append", lib().rolaq_quantize_append(
+        ctypes.byref(d), ctypes.byref(params), _ptr(R_split), _ptr(c), _ptr(k_r), _ptr(req), _ptr(pos),
+        _ptr(seq_lens), n, _stream(stream)))
+
+
+def decode_workspace_bytes(batch: int, heads: int) -> int:
+    return int(lib().rolaq_decode_workspace_bytes(batch, heads))
+
+
+def decode_attn(cache: PagedCache, params: rolaq_layer_params, q_c_rot: torch.Tensor, q_r: torch.Tensor,
+                seq_lens: torch.Tensor, sm_scale: float, out: Optional[torch.Tensor] = None,
+                lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                stream=None):
+    B, H = int(q_c_rot.shape[0]), int(q_c_rot.shape[1])
+    assert q_c_rot.dtype == torch.bfloat16 and q_r.dtype == torch.bfloat16
+    dev = q_c_rot.device
+    if out is None:
+        out = torch.empty((B, H, D_C), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    nbytes = decode_workspace_bytes(B, H)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    d = cache.desc()
+    _check("rolaq_decode_attn", lib().rolaq_decode_attn(
+        ctypes.byref(d), ctypes.byref(params), _ptr(q_c_rot), _ptr(q_r), _ptr(seq_lens), B, H,
+        float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def get_status(stream=None) -> int:
+    v = ctypes.c_int(0)
+    _check("rolaq_get_status", lib().rolaq_get_status(ctypes.byref(v), _stream(stream)))
+    return v.value

@@ -88,6 +88,7 @@ extern "C" {
 /* Device status bits reported by rolaq_get_status(). */
 #define ROLAQ_STATUS_BAD_PAGE   1  /* page-table entry < 0 or >= num_pages (skipped)  */
 #define ROLAQ_STATUS_BAD_SLOT   2  /* append target outside its request's pages       */
+#define ROLAQ_STATUS_TIMEOUT    4  /* a pipeline wait gave up (results of that call invalid) */
 
 /* Cache descriptor.  Plain data; the caller owns every buffer it points to.
  *   pages_dev       page pool, num_pages * ROLAQ_PAGE_BYTES bytes, 1024-B aligned.

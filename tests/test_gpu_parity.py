@@ -1,0 +1,217 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import rolaq_oracle as O
+from decode_attention_rotate_b200 import rolaq as R
+from decode_attention_rotate_b200 import workloads as W
+from tests.gpu_helpers import (DECODE_TOL, META_TOL, SM_SCALE, bf16_bits, build_oracle_cache,
+                               codes_match, f64, meta_match, oracle_decode, rel_l2)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    R.lib()
+    yield
+    assert R.get_status() == 0
+
+
+def _quantize_on_gpu(w, layer, seq_lens, tau, gain, n_sink=0, n_recent=0, zero_latent=False):
+    Rm = W.rotation(w.seed + layer)
+    R_split = R.prepare_rotation(torch.as_tensor(Rm).to(DEV))
+    pt = W.page_table(W.Workload(w.name, len(seq_lens), tuple(seq_lens), w.heads,
+                                 paged_shuffled=w.paged_shuffled, seed=w.seed))
+    num_pages = int(pt.max() + 1)
+    cache = R.PagedCache(num_pages, torch.as_tensor(pt), n_sink, n_recent, device=DEV)
+    cache.pages.fill_(0xAB)                       # unwritten bytes must stay untouched
+    cs, krs, reqs, poss = [], [], [], []
+    for r, L in enumerate(seq_lens):
+        c = W.latent(w, layer, L, stream=100 + r)
+        if zero_latent:
+            c = torch.zeros_like(c)
+        cs.append(c)
+        krs.append(W.rope_key(w, layer, L, stream=200 + r))
+        reqs.append(torch.full((L,), r, dtype=torch.int32))
+        poss.append(torch.arange(L, dtype=torch.int32))
+    c = torch.cat(cs).to(DEV)
+    kr = torch.cat(krs).to(DEV)
+    req = torch.cat(reqs).to(DEV)
+    pos = torch.cat(poss).to(DEV)
+    lens = torch.as_tensor(seq_lens, dtype=torch.int32).to(DEV)
+    p = R.layer_params_init(tau, gain)
+    R.quantize_append(cache, p, R_split, c, kr, req, pos, lens)
+    torch.cuda.synchronize()
+    return cache, cs, krs, Rm.astype(np.float64), pt
+
+
+def _check_write(cache, cs, krs, Rm, pt, seq_lens, tau, gain, n_sink=0, n_recent=0):
+    pool = cache.pages.cpu().numpy()
+    frac_total, n_total = 0.0, 0
+    prot = cache.prot.float().cpu().numpy() if cache.prot is not None else None
+    for r, L in enumerate(seq_lens):
+        if L == 0:
+            continue
+        q = O.quantize(f64(cs[r]), Rm, tau, gain)
+        packed, meta, kr = O.pages_read_fast(pool, pt, r, L)
+        ok, frac, nbad = codes_match(packed, q, tau)
+        assert ok, f"request {r}: {nbad} codes differ outside the threshold window"
+        frac_total += frac * L
+        n_total += L
+        emu, es = meta_match(meta, q, gain)
+        assert emu <= META_TOL and es <= META_TOL, (emu, es)
+        assert (kr == bf16_bits(krs[r])).all()
+        if prot is not None:
+            yb = O.bf16_round(q["y"])
+            for p in range(L):
+                if p < n_sink:
+                    slot = p
+                elif p >= L - n_recent:
+                    slot = n_sink + p % n_recent
+                else:
+                    continue
+                # bf16 of an fp32 y that is within ~1e-6 relative of the fp64 y: at most
+                # one bf16 ulp apart
+                d = np.abs(prot[r, slot] - yb[p])
+                assert (d <= np.abs(yb[p]) * 2.0 ** -7 + 1e-30).all()
+    return frac_total / max(n_total, 1)
+
+
+def test_quantize_tiny():
+    w = W.TINY
+    frac = None
+    cache, cs, krs, Rm, pt = _quantize_on_gpu(w, 0, [256], 0.9816, 1.16)
+    frac = _check_write(cache, cs, krs, Rm, pt, [256], 0.9816, 1.16)
+    assert frac < 1e-3
+
+
+def test_quantize_ragged_multi_request_shuffled_pages():
+    w = W.Workload("ragged", 3, (1, 300, 129), 16, paged_shuffled=True, seed=77)
+    tau, gain = 0.87, 1.07
+    cache, cs, krs, Rm, pt = _quantize_on_gpu(w, 0, [1, 300, 129], tau, gain)
+    _check_write(cache, cs, krs, Rm, pt, [1, 300, 129], tau, gain)
+    # bytes of pages no token was written to are untouched
+    pool = cache.pages.cpu().numpy().reshape(-1, O.PAGE_BYTES)
+    assert (pool[pt[0, 0], 288 * 0 + 128:O.PAGE_META] == 0xAB).all()
+
+
+def test_quantize_protected_side_store():
+    w = W.Workload("prot", 2, (200, 40), 16, seed=78)
+    tau, gain = 1.05, 1.12
+    cache, cs, krs, Rm, pt = _quantize_on_gpu(w, 0, [200, 40], tau, gain, n_sink=4, n_recent=16)
+    _check_write(cache, cs, krs, Rm, pt, [200, 40], tau, gain, 4, 16)
+
+
+def test_quantize_zero_latent_group():
+    w = W.Workload("zero", 1, (70,), 16, seed=79)
+    cache, cs, krs, Rm, pt = _quantize_on_gpu(w, 0, [70], 0.95, 1.1, zero_latent=True)
+    packed, meta, _ = O.pages_read_fast(cache.pages.cpu().numpy(), pt, 0, 70)
+    assert (O.unpack(packed) == 2).all()
+    assert (meta == 0).all()
+
+
+def _decode_case(w, seq_lens, H, tau, gain, n_sink=0, n_recent=0, layer=0):
+    cache, data, Rm = build_oracle_cache(w, layer, seq_lens, tau, gain, n_sink, n_recent)
+    B = len(seq_lens)
+    ww = W.Workload(w.name, B, tuple(seq_lens), H, seed=w.seed)
+    q_c, q_r = W.queries(ww, layer)
+    p = R.layer_params_init(tau, gain)
+    lens = torch.as_tensor(seq_lens, dtype=torch.int32).to(DEV)
+    out, lse = R.decode_attn(cache, p, q_c.to(DEV), q_r.to(DEV), lens, SM_SCALE)
+    torch.cuda.synchronize()
+    o_ref, l_ref = oracle_decode(data, f64(q_c), f64(q_r), seq_lens, tau, SM_SCALE, n_sink, n_recent)
+    out = out.cpu().numpy().astype(np.float64)
+    lse = lse.cpu().numpy().astype(np.float64)
+    for r, L in enumerate(seq_lens):
+        if L == 0:
+            assert (out[r] == 0).all() and np.isneginf(lse[r]).all()
+            continue
+        e = rel_l2(out[r], o_ref[r])
+        assert e.max() <= DECODE_TOL, (r, e.max())
+        assert np.abs(lse[r] - l_ref[r]).max() <= 1e-2 * max(1.0, np.abs(l_ref[r]).max()), r
+    return out, o_ref
+
+
+def test_decode_tiny():
+    _decode_case(W.TINY, [256], 16, 0.9816, 1.16)
+
+
+def test_decode_ragged_lengths_and_empty():
+    w = W.Workload("dr", 5, (1, 63, 64, 65, 0), 16, paged_shuffled=True, seed=90)
+    _decode_case(w, [1, 63, 64, 65, 0], 16, 0.9, 1.05)
+
+
+def test_decode_several_splits():
+    # 3 requests of a few thousand tokens: many split-K items per request
+    w = W.Workload("ds", 3, (4096, 3000, 777), 16, paged_shuffled=True, seed=91)
+    _decode_case(w, [4096, 3000, 777], 16, 0.93, 1.18)
+
+
+def test_decode_128_heads_paged():
+    w = W.Workload("h128", 4, (1024, 2500, 64, 1500), 128, paged_shuffled=True, seed=92)
+    _decode_case(w, [1024, 2500, 64, 1500], 128, 0.88, 1.02)
+
+
+def test_decode_sink_and_recent_protection():
+    w = W.Workload("mix", 3, (1000, 130, 5), 16, seed=93)
+    _decode_case(w, [1000, 130, 5], 16, 0.97, 1.1, n_sink=4, n_recent=128)
+
+
+def test_decode_single_token_equals_its_reconstruction():
+    w = W.Workload("one", 1, (1,), 16, seed=94)
+    out, ref = _decode_case(w, [1], 16, 0.9, 1.0)
+    assert rel_l2(out[0], ref[0]).max() < 5e-3
+
+
+def test_end_to_end_write_then_decode():
+    """Cache written by the GPU write path, decoded on the GPU, against the oracle decoding
+    the GPU-written records."""
+    w = W.Workload("e2e", 2, (700, 1333), 16, paged_shuffled=True, seed=95)
+    tau, gain = 0.91, 1.13
+    lens_l = [700, 1333]
+    cache, cs, krs, Rm, pt = _quantize_on_gpu(w, 0, lens_l, tau, gain, n_sink=4, n_recent=128)
+    q_c, q_r = W.queries(W.Workload("e2e", 2, tuple(lens_l), 16, seed=95), 0)
+    p = R.layer_params_init(tau, gain)
+    lens = torch.as_tensor(lens_l, dtype=torch.int32).to(DEV)
+    out, lse = R.decode_attn(cache, p, q_c.to(DEV), q_r.to(DEV), lens, SM_SCALE)
+    pool = cache.pages.cpu().numpy()
+    prot = cache.prot.float().cpu().numpy().astype(np.float64)
+    for r, L in enumerate(lens_l):
+        packed, meta, kr = O.pages_read_fast(pool, pt, r, L)
+        content = np.zeros((L, 512))
+        for pp in range(L):
+            if pp < 4:
+                content[pp] = prot[r, pp]
+            elif pp >= L - 128:
+                content[pp] = prot[r, 4 + pp % 128]
+        o, l = O.decode_request(f64(q_c[r]), f64(q_r[r]), packed, meta, O.bf16_bits_to_f64(kr), tau,
+                                SM_SCALE, content, 4, 128)
+        e = rel_l2(out[r].cpu().numpy().astype(np.float64), o)
+        assert e.max() <= DECODE_TOL, e.max()
+
+
+def test_bad_page_entry_sets_status_and_skips():
+    w = W.Workload("bad", 1, (256,), 16, seed=96)
+    cache, data, _ = build_oracle_cache(w, 0, [256], 0.9, 1.0)
+    cache.page_table[0, 1] = cache.num_pages + 5          # outside the pool
+    q_c, q_r = W.queries(w, 0)
+    p = R.layer_params_init(0.9, 1.0)
+    lens = torch.tensor([256], dtype=torch.int32, device=DEV)
+    out, _ = R.decode_attn(cache, p, q_c.to(DEV), q_r.to(DEV), lens, SM_SCALE)
+    st = R.get_status()
+    assert st & R.STATUS_BAD_PAGE
+    assert torch.isfinite(out).all()
+    # tokens of the skipped page are left out: compare with the oracle on the other pages
+    keep = np.r_[0:64, 128:256]
+    d = data[0]
+    xq = O.dequantize(d["q"]["packed"], d["q"]["meta"], 0.9)[keep]
+    o_ref, _ = O.attend(f64(q_c[0]), f64(q_r[0]), xq, d["k_r"][keep], SM_SCALE)
+    assert rel_l2(out[0].cpu().numpy().astype(np.float64), o_ref).max() <= DECODE_TOL

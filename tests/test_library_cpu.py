@@ -1,0 +1,98 @@
+"""CPU checks of the C-ABI library: it builds for sm_100a, loads, exports every function
+include/rolaq.h declares, and rejects bad arguments on the host (no kernel launches)."""
+import ctypes
+import math
+import subprocess
+
+import pytest
+
+from decode_attention_rotate_b200 import build as B
+from decode_attention_rotate_b200 import rolaq as R
+from oracle import rolaq_oracle as O
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return R.lib()
+
+
+def test_exports_every_declared_function(lib):
+    names = R.header_functions()
+    assert "rolaq_decode_attn" in names and "rolaq_quantize_append" in names
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_version_and_strerror(lib):
+    assert R.version() == 100
+    assert "workspace" in R.strerror(-2)
+    assert R.strerror(12345) == "unknown error"
+
+
+def test_layer_params_levels_match_oracle(lib):
+    for tau in (0.85, 0.9816, 1.1):
+        p = R.layer_params_init(tau, 1.16)
+        a, b = O.levels(tau)
+        assert p.level_a == pytest.approx(a, rel=1e-7)
+        assert p.level_b == pytest.approx(b, rel=1e-7)
+        assert p.level_a == float(ctypes.c_float(a).value)
+    with pytest.raises(R.RolaqError):
+        R.layer_params_init(0.0, 1.0)
+    with pytest.raises(R.RolaqError):
+        R.layer_params_init(1.0, float("nan"))
+
+
+def _cache(**kw):
+    c = R.rolaq_cache()
+    c.pages_dev = kw.get("pages", 1 << 20)
+    c.num_pages = kw.get("num_pages", 4)
+    c.page_table_dev = kw.get("pt", 1 << 21)
+    c.batch = kw.get("batch", 2)
+    c.max_pages_per_seq = kw.get("max_pages", 2)
+    c.prot_dev = kw.get("prot", None)
+    c.n_sink = kw.get("n_sink", 0)
+    c.n_recent = kw.get("n_recent", 0)
+    return c
+
+
+def test_decode_argument_errors(lib):
+    p = R.rolaq_layer_params(0.9, 1.0, 0.45, 1.5)
+    ptr = 1 << 22
+    def call(cache, heads=16, batch=2, ws=1 << 30, q=ptr):
+        return lib.rolaq_decode_attn(ctypes.byref(cache), ctypes.byref(p), q, ptr, ptr, batch, heads,
+                                     0.07, ptr, ptr, ptr, ws, None)
+    assert call(_cache(pages=None)) == -1
+    assert call(_cache(pages=(1 << 20) + 8)) == -1          # misaligned pool
+    assert call(_cache(), heads=24) == -4
+    assert call(_cache(), heads=0) == -4
+    assert call(_cache(), batch=3) == -1                     # more requests than the cache
+    assert call(_cache(), ws=16) == -2
+    assert call(_cache(), q=None) == -1
+    assert call(_cache(n_sink=4)) == -1                      # protection without a side store
+    bad = R.rolaq_layer_params(0.9, 1.0, 1.5, 0.45)          # levels out of order
+    assert lib.rolaq_decode_attn(ctypes.byref(_cache()), ctypes.byref(bad), ptr, ptr, ptr, 2, 16, 0.07,
+                                 ptr, ptr, ptr, 1 << 30, None) == -1
+
+
+def test_quantize_argument_errors(lib):
+    p = R.rolaq_layer_params(0.9, 1.0, 0.45, 1.5)
+    ptr = 1 << 22
+    def call(cache, n=10, c=ptr, seq=ptr):
+        return lib.rolaq_quantize_append(ctypes.byref(cache), ctypes.byref(p), ptr, c, ptr, ptr, ptr, seq, n, None)
+    assert call(_cache(), n=-1) == -1
+    assert call(_cache(), n=0) == 0
+    assert call(_cache(), c=None) == -1
+    assert call(_cache(), c=ptr + 2) == -1
+    assert call(_cache(n_recent=8, prot=ptr), seq=None) == -1
+
+
+def test_workspace_bytes_shape_rules(lib):
+    assert lib.rolaq_decode_workspace_bytes(4, 24) == 0
+    assert lib.rolaq_decode_workspace_bytes(0, 16) == 0
+    n16 = lib.rolaq_decode_workspace_bytes(4, 16)
+    assert n16 > 0 and n16 % 16 == 0
