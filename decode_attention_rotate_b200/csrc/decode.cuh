@@ -28,6 +28,7 @@ constexpr int kPageRows = ROLAQ_PAGE_BYTES / 128;   // 144 rows of 128 B
 constexpr int kNStage = 8;                          // half-page stages per team
 constexpr int kTStride = 40;                        // floats per head row of sT / sP
 constexpr int kDecodeThreads = 256;
+constexpr float kRescaleLog2 = 8.f;
 // A team stages its half of a page: 32 code rows, 8 metadata rows, 32 RoPE rows.
 constexpr int kHalfBytes = 9216;
 constexpr int kHalfMetaOff = 4096;                  // smem row 32
@@ -44,7 +45,8 @@ struct DecodeArgs {
     const int32_t* seq_lens;
     int batch, heads;
     float scale_log2;            // sm_scale * log2(e)
-    uint32_t lut_lo, lut_hi;     // low / high bytes of the four bf16 levels
+    uint32_t lut_lo, lut_hi;     // low / high bytes of the four bf16 levels / kappa
+    float kappa;                 // level = kappa * bf16 level
     int target_items;
     float* ws_o;                 // [items][2][heads][512]
     float2* ws_ml;               // [items][2][heads]  (running max (log2 units), sum)
@@ -153,6 +155,102 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t lo, uint32_t h
     uint32_t m3 = w & 0xC0C0C0C0u;
     r[3][0] = prmt(lo, hi, __umulhi(m3, 0x11u << 26) + 0x40404040u);
     r[3][1] = prmt(lo, hi, __umulhi(m3, 0x11u << 10) + 0x4040u);
+}
+
+// QK for one team's half page (32 tokens) and one 128-channel group: dequantise the
+// codes into bf16 level fragments (kept in bq for the PV step), run the MMAs, fold the
+// group metadata, add the RoPE part and store the partial scores.  FULL: all 32 tokens
+// are in the sequence and none is protected (no per-token masks).
+template <bool FULL>
+__device__ __forceinline__ void qk_half(const uint8_t* pg, float (*sT)[kTStride], int r, int i, int g,
+                                        uint32_t lut_lo, uint32_t lut_hi, float kappa,
+                                        const uint32_t (&qa)[8][4], const uint32_t (&qra)[4],
+                                        float qs0, float qs1, int nvalid, int pos0, int L,
+                                        int recent_start, const DecodeArgs& args, int b,
+                                        uint32_t (&bq)[4][8][2], float (&mu)[4][2], float (&sc)[4][2]) {
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        const uint2 w = *reinterpret_cast<const uint2*>(pg + swz128(8 * nt + r, 32 * g + 8 * i));
+        uint32_t t[4][2];
+        dequant_word(w.x, lut_lo, lut_hi, t);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) { bq[nt][kk][0] = t[kk][0]; bq[nt][kk][1] = t[kk][1]; }
+        dequant_word(w.y, lut_lo, lut_hi, t);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) { bq[nt][4 + kk][0] = t[kk][0]; bq[nt][4 + kk][1] = t[kk][1]; }
+    }
+    if (!FULL) {
+        // Protected tokens read their bf16 rotated content instead of the codes.
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const int pos = pos0 + 8 * nt + r;
+            if (pos < L && (pos < args.n_sink || pos >= recent_start)) {
+                const int slot = pos < args.n_sink ? pos : args.n_sink + pos % args.n_recent;
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    args.prot + ((size_t)b * (args.n_sink + args.n_recent) + slot) * ROLAQ_D_C + 128 * g + 32 * i);
+                uint32_t wv[16];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint4 v = src[q4];
+                    wv[4 * q4 + 0] = v.x; wv[4 * q4 + 1] = v.y; wv[4 * q4 + 2] = v.z; wv[4 * q4 + 3] = v.w;
+                }
+#pragma unroll
+                for (int s = 0; s < 8; ++s) {
+                    const int base = 16 * (s >> 2), kk = s & 3;
+                    const uint32_t sel = (kk & 1) ? 0x7632u : 0x5410u;
+                    bq[nt][s][0] = prmt(wv[(base + kk) >> 1], wv[(base + 4 + kk) >> 1], sel);
+                    bq[nt][s][1] = prmt(wv[(base + 8 + kk) >> 1], wv[(base + 12 + kk) >> 1], sel);
+                }
+            }
+        }
+    }
+    // metadata of the two tokens in each n-tile column pair: mean, scale (kappa folded in)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int t = 8 * nt + 2 * i + e;               // token row in the half
+            const float2 ms = *reinterpret_cast<const float2*>(pg + swz128(32 + (t >> 2), (t & 3) * 32 + 8 * g));
+            if (FULL) {
+                mu[nt][e] = ms.x;
+                sc[nt][e] = ms.y * kappa;
+            } else {
+                const int pos = pos0 + t;
+                const bool valid = t < nvalid;
+                const bool prot = pos < args.n_sink || pos >= recent_start;
+                mu[nt][e] = (valid && !prot) ? ms.x : 0.f;
+                sc[nt][e] = valid ? (prot ? 1.f : ms.y * kappa) : 0.f;
+            }
+        }
+    float acc[4][4];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) mma_bf16_16816(acc[nt], qa[s], bq[nt][s][0], bq[nt][s][1]);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        // fold the group metadata: q.x = mean * sum(q_g) + scale * (q_g . level)
+        acc[nt][0] = fmaf(sc[nt][0], acc[nt][0], mu[nt][0] * qs0);
+        acc[nt][1] = fmaf(sc[nt][1], acc[nt][1], mu[nt][1] * qs0);
+        acc[nt][2] = fmaf(sc[nt][0], acc[nt][2], mu[nt][0] * qs1);
+        acc[nt][3] = fmaf(sc[nt][1], acc[nt][3], mu[nt][1] * qs1);
+        // RoPE part of the score for channels 16g..16g+15
+        const int row = 40 + 8 * nt + r;
+        const uint32_t kb0 = *reinterpret_cast<const uint32_t*>(pg + swz128(row, 32 * g + 4 * i));
+        const uint32_t kb1 = *reinterpret_cast<const uint32_t*>(pg + swz128(row, 32 * g + 16 + 4 * i));
+        mma_bf16_16816(acc[nt], qra, kb0, kb1);
+        const int tl = 8 * nt + 2 * i;
+        if (!FULL) {
+            if (tl >= nvalid) { acc[nt][0] = -INFINITY; acc[nt][2] = -INFINITY; }
+            if (tl + 1 >= nvalid) { acc[nt][1] = -INFINITY; acc[nt][3] = -INFINITY; }
+        }
+        *reinterpret_cast<float2*>(&sT[r][tl]) = make_float2(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<float2*>(&sT[r + 8][tl]) = make_float2(acc[nt][2], acc[nt][3]);
+    }
 }
 
 // Issue the three copies of one team's half of page `k` (or mark it invalid).
@@ -284,87 +382,14 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map32, const __grid_const
         } else {
             const uint8_t* pg = sm.stage[team][st];
             const bool mixed = protect && (pos0 < args.n_sink || pos0 + 32 > recent_start);
-
-            // ---- QK: dequantised level fragments for 4 n-tiles of 8 tokens -------
             uint32_t bq[4][8][2];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const uint2 w = *reinterpret_cast<const uint2*>(pg + swz128(8 * nt + r, 32 * g + 8 * i));
-                uint32_t t[4][2];
-                dequant_word(w.x, lut_lo, lut_hi, t);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) { bq[nt][kk][0] = t[kk][0]; bq[nt][kk][1] = t[kk][1]; }
-                dequant_word(w.y, lut_lo, lut_hi, t);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) { bq[nt][4 + kk][0] = t[kk][0]; bq[nt][4 + kk][1] = t[kk][1]; }
-            }
-            if (mixed) {
-                // Protected tokens read their bf16 rotated content instead of the codes.
-#pragma unroll
-                for (int nt = 0; nt < 4; ++nt) {
-                    const int pos = pos0 + 8 * nt + r;
-                    if (pos < L && (pos < args.n_sink || pos >= recent_start)) {
-                        const int slot = pos < args.n_sink ? pos : args.n_sink + pos % args.n_recent;
-                        const uint4* src = reinterpret_cast<const uint4*>(
-                            args.prot + ((size_t)b * (args.n_sink + args.n_recent) + slot) * ROLAQ_D_C
-                            + 128 * g + 32 * i);
-                        uint32_t wv[16];
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            uint4 v = src[q4];
-                            wv[4 * q4 + 0] = v.x; wv[4 * q4 + 1] = v.y;
-                            wv[4 * q4 + 2] = v.z; wv[4 * q4 + 3] = v.w;
-                        }
-#pragma unroll
-                        for (int s = 0; s < 8; ++s) {
-                            const int base = 16 * (s >> 2), kk = s & 3;
-                            const uint32_t sel = (kk & 1) ? 0x7632u : 0x5410u;
-                            bq[nt][s][0] = prmt(wv[(base + kk) >> 1], wv[(base + 4 + kk) >> 1], sel);
-                            bq[nt][s][1] = prmt(wv[(base + 8 + kk) >> 1], wv[(base + 12 + kk) >> 1], sel);
-                        }
-                    }
-                }
-            }
-
-            // metadata of the two tokens in each n-tile column pair: mean, scale
             float mu[4][2], sc[4][2];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int t = 8 * nt + 2 * i + e;               // token row in the half
-                    const float2 ms = *reinterpret_cast<const float2*>(
-                        pg + swz128(32 + (t >> 2), (t & 3) * 32 + 8 * g));
-                    const int pos = pos0 + 8 * nt + 2 * i + e;
-                    const bool valid = (8 * nt + 2 * i + e) < nvalid;
-                    const bool prot = mixed && (pos < args.n_sink || pos >= recent_start);
-                    mu[nt][e] = (valid && !prot) ? ms.x : 0.f;
-                    sc[nt][e] = valid ? (prot ? 1.f : ms.y) : 0.f;
-                }
-
-            float acc[4][4];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
-#pragma unroll
-                for (int s = 0; s < 8; ++s) mma_bf16_16816(acc[nt], qa[s], bq[nt][s][0], bq[nt][s][1]);
-                // fold the group metadata: q.x = mean * sum(q_g) + scale * (q_g . level)
-                acc[nt][0] = fmaf(sc[nt][0], acc[nt][0], mu[nt][0] * qs0);
-                acc[nt][1] = fmaf(sc[nt][1], acc[nt][1], mu[nt][1] * qs0);
-                acc[nt][2] = fmaf(sc[nt][0], acc[nt][2], mu[nt][0] * qs1);
-                acc[nt][3] = fmaf(sc[nt][1], acc[nt][3], mu[nt][1] * qs1);
-                // RoPE part of the score for channels 16g..16g+15
-                const int row = 40 + 8 * nt + r;
-                const uint32_t kb0 = *reinterpret_cast<const uint32_t*>(pg + swz128(row, 32 * g + 4 * i));
-                const uint32_t kb1 = *reinterpret_cast<const uint32_t*>(pg + swz128(row, 32 * g + 16 + 4 * i));
-                mma_bf16_16816(acc[nt], qra, kb0, kb1);
-                const int tl = 8 * nt + 2 * i;
-                if (tl >= nvalid) { acc[nt][0] = -INFINITY; acc[nt][2] = -INFINITY; }
-                if (tl + 1 >= nvalid) { acc[nt][1] = -INFINITY; acc[nt][3] = -INFINITY; }
-                *reinterpret_cast<float2*>(&sm.sT[team][g][r][tl]) = make_float2(acc[nt][0], acc[nt][1]);
-                *reinterpret_cast<float2*>(&sm.sT[team][g][r + 8][tl]) = make_float2(acc[nt][2], acc[nt][3]);
-            }
+            if (nvalid == 32 && !mixed)
+                qk_half<true>(pg, sm.sT[team][g], r, i, g, lut_lo, lut_hi, args.kappa, qa, qra, qs0, qs1,
+                              32, pos0, L, recent_start, args, b, bq, mu, sc);
+            else
+                qk_half<false>(pg, sm.sT[team][g], r, i, g, lut_lo, lut_hi, args.kappa, qa, qra, qs0, qs1,
+                               nvalid, pos0, L, recent_start, args, b, bq, mu, sc);
             named_bar_sync(1 + team, 128);
             // every warp of the team is done reading this stage: refill it
             if (producer && k + kNStage < n_pages)
@@ -385,9 +410,13 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map32, const __grid_const
                 pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 1));
                 pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 2));
                 pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 4));
-                const float m_new = fmaxf(m_run, pm);
+                // The reference max moves only when the page max exceeds it by more than
+                // kRescaleLog2 (or on the first finite score), so O is rarely rescaled; the
+                // probabilities relative to a stale reference stay below 2^kRescaleLog2.
+                float m_new = m_run;
+                if (pm > m_run + kRescaleLog2 || m_run == -INFINITY) m_new = pm;
                 const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-                const float alpha = ex2(m_run - m_use);
+                const float alpha = (m_new == m_run) ? 1.f : ex2(m_run - m_use);
                 float4 p;
                 p.x = ex2(sv[0] - m_use); p.y = ex2(sv[1] - m_use);
                 p.z = ex2(sv[2] - m_use); p.w = ex2(sv[3] - m_use);

@@ -3,31 +3,33 @@
 // packing, (mean, gain*std) metadata, the bf16 RoPE key copy and, for protected tokens,
 // bf16(y) into the side store.
 //
-// rolaq_quantize_kernel is persistent (one CTA per SM).  A tile is 128 tokens; it is
-// produced as two halves of 256 output coordinates (two groups each).  Warp roles:
-//   warp 8   producer: bulk tensor copies of c (128 x 32) and of both R planes
-//            (256 x 32 each) per 32-wide K step into a 4-deep shared-memory ring;
-//   warp 9   allocates 512 TMEM columns and issues tcgen05.mma (M=128, N=256, K=16,
-//            bf16 in, fp32 accumulate) for R_hi and R_lo into one accumulator, so
-//            y = c.R_hi + c.R_lo carries ~2^-17 relative error; the two halves use
-//            separate accumulators (TMEM columns 0..255 / 256..511), so the epilogue
-//            of one half overlaps the MMAs of the next;
-//   warps 0..7  epilogue: warp e reads TMEM lanes 32*(e%4).. (one token per thread) and
-//            quantizes group 2*half + e/4 of that token.
+// rolaq_quantize_kernel is persistent (one CTA per SM).  A tile is 128 tokens (the TMEM
+// lanes); its c block stays in shared memory while the four groups of 128 output
+// coordinates are produced one after the other (one job per group).  Warp roles:
+//   warp 8      producer: bulk tensor copies of the c tile (16 chunks of 128 x 32) and
+//               of the R-plane chunks (128 x 32) each job needs;
+//   warp 9      allocates 512 TMEM columns and issues tcgen05.mma (M=128, N=128, K=16,
+//               bf16 in, fp32 accumulate).  R = R_hi + R_mid + R_lo (three bf16 planes,
+//               ~2^-26 relative).  The tensor cores truncate each fp32 accumulation step
+//               toward zero, so a job keeps two accumulators: chain A takes R_lo and R_mid
+//               over all of K first (while it is small) and then R_hi over K < 256, chain B
+//               takes R_hi over K >= 256; y = A + B.  That bounds the bias to 16 large
+//               truncations per chain.  Jobs alternate between two TMEM buffers, so the
+//               epilogue of one group overlaps the MMAs of the next;
+//   warps 0..7  epilogue in two sets of four; set e quantizes groups e and e + 2.
 #pragma once
 #include "common.cuh"
 
 namespace rolaq {
 
-constexpr int kQTileM = 128;
-constexpr int kQHalfN = 256;
-constexpr int kQK = 32;                       // K per stage (64-byte rows, 64B swizzle)
-constexpr int kQStages = 4;
+constexpr int kQTileM = 128;                  // tokens per tile (TMEM lanes)
+constexpr int kQN = ROLAQ_GROUP;              // output coordinates per job: one group
+constexpr int kQK = 32;                       // K per chunk (64-byte rows, 64B swizzle)
 constexpr int kQKSteps = ROLAQ_D_C / kQK;     // 16
+constexpr int kQStages = 5;
 constexpr int kQThreads = 320;
-constexpr uint32_t kQStageABytes = kQTileM * kQK * 2;     // 8 KB
-constexpr uint32_t kQStageBBytes = kQHalfN * kQK * 2;     // 16 KB per plane
-constexpr uint32_t kQStageTx = kQStageABytes + 2 * kQStageBBytes;
+constexpr int kQPlanes = 3;
+constexpr uint32_t kQChunkBytes = kQTileM * kQK * 2;      // 8 KB (c chunk or one R-plane chunk)
 
 struct QuantArgs {
     uint8_t* pages;
@@ -45,10 +47,11 @@ struct QuantArgs {
 };
 
 struct QuantSmem {
-    alignas(1024) uint8_t a[kQStages][kQStageABytes];
-    alignas(1024) uint8_t bh[kQStages][kQStageBBytes];
-    alignas(1024) uint8_t bl[kQStages][kQStageBBytes];
-    alignas(8) uint64_t full[kQStages];
+    alignas(1024) uint8_t a[kQKSteps][kQChunkBytes];        // resident c tile, 16 K chunks
+    alignas(1024) uint8_t b[kQStages][2][kQChunkBytes];     // streamed R-plane chunks
+    alignas(8) uint64_t a_full[kQKSteps];
+    uint64_t a_free[kQKSteps];
+    uint64_t full[kQStages];
     uint64_t empty[kQStages];
     uint64_t tfull[2];
     uint64_t tempty[2];
@@ -62,8 +65,8 @@ __device__ __forceinline__ uint64_t umma_desc_sw64(uint32_t saddr) {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (32ull << 32) | (1ull << 46) |
            (4ull << 61);
 }
-// Instruction descriptor: bf16 x bf16 -> f32, both K-major, M = 128, N = 256.
-constexpr uint32_t kQIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kQHalfN >> 3) << 17) |
+// Instruction descriptor: bf16 x bf16 -> f32, both K-major, M = 128, N = 128.
+constexpr uint32_t kQIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kQN >> 3) << 17) |
                              ((uint32_t)(kQTileM >> 4) << 24);
 
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t acc) {
@@ -99,33 +102,40 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-
-// Quantize one 128-coordinate group of one token straight from TMEM (this thread's
-// lane, columns col..col+127), streaming 32 columns at a time in three passes: mean,
-// population std, then codes (and the bf16 copy for a protected token).  All lanes of
-// the warp must call it (the TMEM loads are warp-wide); `store` is false for lanes
-// without a valid target.
-__device__ __forceinline__ void quantize_group_tmem(uint32_t col, float tau, float gain, bool store,
-                                                    uint8_t* dst_codes, float* dst_meta,
-                                                    __nv_bfloat16* dst_prot) {
+// 32 columns of y = chain A + chain B (fp32 add of the two K-half accumulators).
+__device__ __forceinline__ void load_y32(uint32_t col_a, uint32_t col_b, float (&y)[32]) {
     float t[32];
+    tmem_ld32(col_a, y);
+    tmem_ld32(col_b, t);
+    tmem_ld_wait();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) y[j] += t[j];
+}
+
+// Quantize one 128-coordinate group of one token straight from TMEM (this thread's lane;
+// chain A at col_a.., chain B at col_b..), streaming 32 columns at a time in three
+// passes: mean, population std, then codes (and the bf16 copy for a protected token).
+// All lanes of the warp must call it (the TMEM loads are warp-wide); `store` is false for
+// lanes without a valid target.
+__device__ __forceinline__ void quantize_group_tmem(uint32_t col_a, uint32_t col_b, float tau, float gain,
+                                                    bool store, uint8_t* dst_codes, float* dst_meta,
+                                                    __nv_bfloat16* dst_prot) {
+    float y[32];
     float s = 0.f;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
-        tmem_ld32(col + 32 * c, t);
-        tmem_ld_wait();
+        load_y32(col_a + 32 * c, col_b + 32 * c, y);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) s += t[j];
+        for (int j = 0; j < 32; ++j) s += y[j];
     }
     const float mean = s * (1.f / 128.f);
     float ss = 0.f;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
-        tmem_ld32(col + 32 * c, t);
-        tmem_ld_wait();
+        load_y32(col_a + 32 * c, col_b + 32 * c, y);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-            const float d = t[j] - mean;
+            const float d = y[j] - mean;
             ss = fmaf(d, d, ss);
         }
     }
@@ -135,14 +145,13 @@ __device__ __forceinline__ void quantize_group_tmem(uint32_t col, float tau, flo
     uint32_t w[8];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-        tmem_ld32(col + 32 * c, t);
-        tmem_ld_wait();
+        load_y32(col_a + 32 * c, col_b + 32 * c, y);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             uint32_t acc = 0;
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const float z = (t[16 * h + j] - mean) * inv;
+                const float z = (y[16 * h + j] - mean) * inv;
                 const uint32_t code = (uint32_t)(z >= -tau) + (uint32_t)(z >= 0.f) + (uint32_t)(z >= tau);
                 acc |= code << (2 * j);
             }
@@ -152,8 +161,8 @@ __device__ __forceinline__ void quantize_group_tmem(uint32_t col, float tau, flo
             uint4* dp = reinterpret_cast<uint4*>(dst_prot + 32 * c);
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8)
-                dp[q8] = make_uint4(pack_bf16(t[8 * q8 + 0], t[8 * q8 + 1]), pack_bf16(t[8 * q8 + 2], t[8 * q8 + 3]),
-                                    pack_bf16(t[8 * q8 + 4], t[8 * q8 + 5]), pack_bf16(t[8 * q8 + 6], t[8 * q8 + 7]));
+                dp[q8] = make_uint4(pack_bf16(y[8 * q8 + 0], y[8 * q8 + 1]), pack_bf16(y[8 * q8 + 2], y[8 * q8 + 3]),
+                                    pack_bf16(y[8 * q8 + 4], y[8 * q8 + 5]), pack_bf16(y[8 * q8 + 6], y[8 * q8 + 7]));
         }
     }
     if (store) {
@@ -174,13 +183,17 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
     const int n_tiles = (args.n + kQTileM - 1) / kQTileM;
 
     if (threadIdx.x == 0) {
+        for (int k = 0; k < kQKSteps; ++k) {
+            mbar_init(smem_u32(&sm.a_full[k]), 1);
+            mbar_init(smem_u32(&sm.a_free[k]), 1);
+        }
         for (int s = 0; s < kQStages; ++s) {
             mbar_init(smem_u32(&sm.full[s]), 1);
             mbar_init(smem_u32(&sm.empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&sm.tfull[a]), 1);
-            mbar_init(smem_u32(&sm.tempty[a]), 8);
+            mbar_init(smem_u32(&sm.tempty[a]), 4);
         }
         sm.abort = 0;
         fence_mbar_init();
@@ -198,99 +211,138 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
 
     if (warp == 8) {
         // ------------------------------------------------------------- producer --
+        // Per tile: the 16 c chunks (once, kept for all four groups) and, per group, the
+        // R_lo/R_mid chunks of the first pass then the R_hi chunks of the second.
         if (lane == 0) {
             uint32_t it = 0;
+            int tl = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x)
-                for (int nh = 0; nh < 2 && ok; ++nh)
-                    for (int kc = 0; kc < kQKSteps; ++kc, ++it) {
-                        const int st = it % kQStages;
-                        if (it >= kQStages && !mbar_wait(smem_u32(&sm.empty[st]), ((it / kQStages) - 1) & 1, &sm.abort)) {
-                            ok = false;
-                            break;
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tl)
+                for (int g = 0; g < ROLAQ_GROUPS && ok; ++g)
+                    for (int pass = 0; pass < 2 && ok; ++pass)
+                        for (int kc = 0; kc < kQKSteps; ++kc, ++it) {
+                            if (g == 0 && pass == 0) {
+                                if (tl > 0 && !mbar_wait(smem_u32(&sm.a_free[kc]), (tl - 1) & 1, &sm.abort)) {
+                                    ok = false;
+                                    break;
+                                }
+                                mbar_arrive_expect_tx(smem_u32(&sm.a_full[kc]), kQChunkBytes);
+                                tma_load_2d(smem_u32(sm.a[kc]), &map_c, kc * kQK, tile * kQTileM,
+                                            smem_u32(&sm.a_full[kc]));
+                            }
+                            const int st = it % kQStages;
+                            if (it >= kQStages &&
+                                !mbar_wait(smem_u32(&sm.empty[st]), ((it / kQStages) - 1) & 1, &sm.abort)) {
+                                ok = false;
+                                break;
+                            }
+                            const uint32_t fb = smem_u32(&sm.full[st]);
+                            const int n0 = g * kQN;
+                            if (pass == 0) {    // R_lo and R_mid (planes 2, 1)
+                                mbar_arrive_expect_tx(fb, 2 * kQChunkBytes);
+                                tma_load_2d(smem_u32(sm.b[st][0]), &map_r, kc * kQK, 2 * ROLAQ_D_C + n0, fb);
+                                tma_load_2d(smem_u32(sm.b[st][1]), &map_r, kc * kQK, ROLAQ_D_C + n0, fb);
+                            } else {            // R_hi (plane 0)
+                                mbar_arrive_expect_tx(fb, kQChunkBytes);
+                                tma_load_2d(smem_u32(sm.b[st][0]), &map_r, kc * kQK, n0, fb);
+                            }
                         }
-                        const uint32_t fb = smem_u32(&sm.full[st]);
-                        mbar_arrive_expect_tx(fb, kQStageTx);
-                        tma_load_2d(smem_u32(sm.a[st]), &map_c, kc * kQK, tile * kQTileM, fb);
-                        tma_load_2d(smem_u32(sm.bh[st]), &map_r, kc * kQK, nh * kQHalfN, fb);
-                        tma_load_2d(smem_u32(sm.bl[st]), &map_r, kc * kQK, ROLAQ_D_C + nh * kQHalfN, fb);
-                    }
         }
     } else if (warp == 9) {
         // ----------------------------------------------------------------- MMA ----
+        // Chain A (TMEM columns buf*256 .. +127): R_lo and R_mid over all of K, then R_hi
+        // over K < 256.  Chain B (+128 .. +255): R_hi over K >= 256.  y = A + B.
         if (lane == 0) {
             uint32_t it = 0, job = 0;
+            int tl = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x)
-                for (int nh = 0; nh < 2 && ok; ++nh, ++job) {
-                    const uint32_t use = job >> 1;
-                    if (use >= 1 && !mbar_wait(smem_u32(&sm.tempty[nh]), (use - 1) & 1, &sm.abort)) { ok = false; break; }
+            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tl)
+                for (int g = 0; g < ROLAQ_GROUPS && ok; ++g, ++job) {
+                    const uint32_t buf = job & 1, use = job >> 1;
+                    if (use >= 1 && !mbar_wait(smem_u32(&sm.tempty[buf]), (use - 1) & 1, &sm.abort)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t d = tmem + (uint32_t)(nh * kQHalfN);
-                    for (int kc = 0; kc < kQKSteps; ++kc, ++it) {
-                        const int st = it % kQStages;
-                        if (!mbar_wait(smem_u32(&sm.full[st]), (it / kQStages) & 1, &sm.abort)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint32_t sa = smem_u32(sm.a[st]);
-                        const uint32_t sbh = smem_u32(sm.bh[st]), sbl = smem_u32(sm.bl[st]);
+                    const uint32_t d_a = tmem + buf * 2 * kQN, d_b = d_a + kQN;
+                    for (int pass = 0; pass < 2 && ok; ++pass)
+                        for (int kc = 0; kc < kQKSteps; ++kc, ++it) {
+                            if (g == 0 && pass == 0 &&
+                                !mbar_wait(smem_u32(&sm.a_full[kc]), tl & 1, &sm.abort)) { ok = false; break; }
+                            const int st = it % kQStages;
+                            if (!mbar_wait(smem_u32(&sm.full[st]), (it / kQStages) & 1, &sm.abort)) { ok = false; break; }
+                            tc_fence_after();
+                            const uint32_t sa = smem_u32(sm.a[kc]);
+                            const uint32_t sb0 = smem_u32(sm.b[st][0]), sb1 = smem_u32(sm.b[st][1]);
 #pragma unroll
-                        for (int k16 = 0; k16 < 2; ++k16) {
-                            const uint64_t da = umma_desc_sw64(sa + 32 * k16);
-                            umma_bf16(d, da, umma_desc_sw64(sbh + 32 * k16), (kc | k16) != 0);
-                            umma_bf16(d, da, umma_desc_sw64(sbl + 32 * k16), 1u);
+                            for (int k16 = 0; k16 < 2; ++k16) {
+                                const uint64_t da = umma_desc_sw64(sa + 32 * k16);
+                                const uint64_t db0 = umma_desc_sw64(sb0 + 32 * k16);
+                                if (pass == 0) {
+                                    umma_bf16(d_a, da, db0, (kc | k16) != 0);
+                                    umma_bf16(d_a, da, umma_desc_sw64(sb1 + 32 * k16), 1u);
+                                } else if (kc < kQKSteps / 2) {
+                                    umma_bf16(d_a, da, db0, 1u);
+                                } else {
+                                    umma_bf16(d_b, da, db0, (kc > kQKSteps / 2 || k16 > 0) ? 1u : 0u);
+                                }
+                            }
+                            umma_commit(smem_u32(&sm.empty[st]));
+                            if (g == ROLAQ_GROUPS - 1 && pass == 1) umma_commit(smem_u32(&sm.a_free[kc]));
                         }
-                        umma_commit(smem_u32(&sm.empty[st]));
-                    }
-                    if (ok) umma_commit(smem_u32(&sm.tfull[nh]));
+                    if (ok) umma_commit(smem_u32(&sm.tfull[buf]));
                 }
         }
     } else {
         // ------------------------------------------------------------ epilogue ----
-        const int q = warp & 3, gg = warp >> 2;
+        // Two sets of four warps take alternate groups (set e: groups e and e + 2, TMEM
+        // buffer e); warp q of a set reads TMEM lanes 32q.. (one token per thread).
+        const int q = warp & 3, set = warp >> 2;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        uint32_t job = 0;
-        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x)
-            for (int nh = 0; nh < 2; ++nh, ++job) {
-                const bool got = mbar_wait(smem_u32(&sm.tfull[nh]), (job >> 1) & 1, &sm.abort);
+        uint32_t use = 0;
+        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            // Target slot of this thread's token, looked up before the accumulator is ready
+            // so the dependent global loads overlap the MMAs.
+            const int tok = tile * kQTileM + 32 * q + lane;
+            long long pid = -1;
+            int rq = -1, ps = 0;
+            if (tok < args.n) {
+                rq = args.req[tok];
+                ps = args.pos[tok];
+                if (rq >= 0 && rq < args.batch && ps >= 0 && (ps / ROLAQ_PAGE_TOKENS) < args.max_pages) {
+                    pid = args.page_table[(long long)rq * args.max_pages + ps / ROLAQ_PAGE_TOKENS];
+                    if (pid >= args.num_pages) pid = -1;
+                }
+                if (pid < 0 && set == 0) raise_status(ROLAQ_STATUS_BAD_SLOT);
+            }
+            const bool store = pid >= 0;
+            uint8_t* page = args.pages + (store ? pid : 0) * (long long)ROLAQ_PAGE_BYTES;
+            const int row = ps % ROLAQ_PAGE_TOKENS;
+            long long prot_row = -1;                  // side-store row of a protected token
+            if (store && args.prot) {
+                const int nslot = args.n_sink + args.n_recent;
+                if (ps < args.n_sink)
+                    prot_row = (long long)rq * nslot + ps;
+                else if (args.n_recent > 0 && ps >= args.seq_lens[rq] - args.n_recent)
+                    prot_row = (long long)rq * nslot + args.n_sink + ps % args.n_recent;
+            }
+            if (store && set == 0) {
+                const uint4* src = reinterpret_cast<const uint4*>(args.k_r + (size_t)tok * ROLAQ_D_R);
+                uint4* dst = reinterpret_cast<uint4*>(page + ROLAQ_PAGE_KR_OFFSET + row * ROLAQ_KR_BYTES);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) dst[j] = src[j];
+            }
+            for (int g = set; g < ROLAQ_GROUPS; g += 2, ++use) {
+                const bool got = mbar_wait(smem_u32(&sm.tfull[set]), use & 1, &sm.abort);
                 tc_fence_after();
-                const int tok = tile * kQTileM + 32 * q + lane;
-                const int g = 2 * nh + gg;
-                long long pid = -1;
-                int rq = -1, ps = 0;
-                if (got && tok < args.n) {
-                    rq = args.req[tok];
-                    ps = args.pos[tok];
-                    if (rq >= 0 && rq < args.batch && ps >= 0 && (ps / ROLAQ_PAGE_TOKENS) < args.max_pages) {
-                        pid = args.page_table[(long long)rq * args.max_pages + ps / ROLAQ_PAGE_TOKENS];
-                        if (pid >= args.num_pages) pid = -1;
-                    }
-                    if (pid < 0 && nh == 0 && gg == 0) raise_status(ROLAQ_STATUS_BAD_SLOT);
-                }
-                const bool store = pid >= 0;
-                uint8_t* page = args.pages + (store ? pid : 0) * (long long)ROLAQ_PAGE_BYTES;
-                const int row = ps % ROLAQ_PAGE_TOKENS;
-                __nv_bfloat16* prot = nullptr;
-                if (store && args.prot) {
-                    const int nslot = args.n_sink + args.n_recent;
-                    if (ps < args.n_sink)
-                        prot = args.prot + ((size_t)rq * nslot + ps) * ROLAQ_D_C + 128 * g;
-                    else if (args.n_recent > 0 && ps >= args.seq_lens[rq] - args.n_recent)
-                        prot = args.prot + ((size_t)rq * nslot + args.n_sink + ps % args.n_recent) * ROLAQ_D_C + 128 * g;
-                }
-                quantize_group_tmem(tmem + lane_base + (uint32_t)(nh * kQHalfN + gg * 128), args.tau, args.gain,
-                                    store, page + ROLAQ_PAGE_CODES_OFFSET + row * ROLAQ_CODE_BYTES + 32 * g,
+                __nv_bfloat16* prot = prot_row >= 0 ? args.prot + prot_row * ROLAQ_D_C + 128 * g : nullptr;
+                const uint32_t col = tmem + lane_base + (uint32_t)(set * 2 * kQN);
+                quantize_group_tmem(col, col + kQN, args.tau, args.gain, store && got,
+                                    page + ROLAQ_PAGE_CODES_OFFSET + row * ROLAQ_CODE_BYTES + 32 * g,
                                     reinterpret_cast<float*>(page + ROLAQ_PAGE_META_OFFSET + row * ROLAQ_META_BYTES) + 2 * g,
                                     prot);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[nh]));
-                if (store && nh == 0 && gg == 0) {
-                    const uint4* src = reinterpret_cast<const uint4*>(args.k_r + (size_t)tok * ROLAQ_D_R);
-                    uint4* dst = reinterpret_cast<uint4*>(page + ROLAQ_PAGE_KR_OFFSET + row * ROLAQ_KR_BYTES);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) dst[j] = src[j];
-                }
+                if (lane == 0) mbar_arrive(smem_u32(&sm.tempty[set]));
             }
+        }
     }
 
     tc_fence_before();
@@ -301,16 +353,20 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
     }
 }
 
-// R (fp32 [512 in][512 out], y = c . R) -> two bf16 planes [2][512 out][512 in]: the
-// nearest bf16 of R^T and the nearest bf16 of the remainder.
+// R (fp32 [512 in][512 out], y = c . R) -> three bf16 planes [3][512 out][512 in]: the
+// nearest bf16 of R^T, of the remainder, and of what remains after that.
 __global__ void rolaq_split_rotation(const float* __restrict__ R, __nv_bfloat16* __restrict__ out) {
     const int o = blockIdx.x;                  // output coordinate (row of R^T)
+    const size_t plane = (size_t)ROLAQ_D_C * ROLAQ_D_C;
     for (int k = threadIdx.x; k < ROLAQ_D_C; k += blockDim.x) {
         const float x = R[(size_t)k * ROLAQ_D_C + o];
         const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+        const float r1 = x - __bfloat162float(hi);
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
         out[(size_t)o * ROLAQ_D_C + k] = hi;
-        out[(size_t)ROLAQ_D_C * ROLAQ_D_C + (size_t)o * ROLAQ_D_C + k] = lo;
+        out[plane + (size_t)o * ROLAQ_D_C + k] = mid;
+        out[2 * plane + (size_t)o * ROLAQ_D_C + k] = lo;
     }
 }
 

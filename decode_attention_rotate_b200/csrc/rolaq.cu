@@ -75,6 +75,31 @@ uint16_t bf16_bits(float x) {
     return (uint16_t)(u >> 16);
 }
 
+// bf16 level pair for the decode MMAs.  Plain bf16(a), bf16(b) are off by up to 2^-9,
+// which moves every score by that much.  Instead pick B = 1 + m/128 and A = bf16(B a/b)
+// over the 128 mantissas m so that A / B matches a / b (typically to ~1e-5; near
+// a/b = 1/4 the choices alias and it degrades to ~1e-3), and return kappa, the
+// geometric mean of a/A and b/B, which splits the remaining ratio error evenly between
+// the two levels.  kappa is folded into the per-token scale.
+void level_encoding(float a, float b, uint16_t* a_bits, uint16_t* b_bits, float* kappa) {
+    const double rho = (double)a / (double)b;
+    double best = 1e30;
+    for (int m = 0; m < 128; ++m) {
+        const double B = 1.0 + m / 128.0;
+        const uint16_t ab = bf16_bits((float)(rho * B));
+        uint32_t u = (uint32_t)ab << 16;
+        float A;
+        memcpy(&A, &u, 4);
+        const double err = fabs((double)A / B - rho);
+        if (err < best) {
+            best = err;
+            *a_bits = ab;
+            *b_bits = bf16_bits((float)B);
+            *kappa = (float)sqrt(((double)a / A) * ((double)b / B));
+        }
+    }
+}
+
 int check_cache(const rolaq_cache* c) {
     if (!c || !c->pages_dev || !c->page_table_dev || c->num_pages <= 0 || c->batch <= 0 ||
         c->max_pages_per_seq <= 0)
@@ -169,7 +194,7 @@ int rolaq_quantize_append(const rolaq_cache* cache, const rolaq_layer_params* p,
     if (!encode_2d(&map_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(c_dev), ROLAQ_D_C,
                    (uint64_t)n, ROLAQ_D_C * 2, kQK, kQTileM, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !encode_2d(&map_r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(R_split_dev), ROLAQ_D_C,
-                   2 * ROLAQ_D_C, ROLAQ_D_C * 2, kQK, kQHalfN, CU_TENSOR_MAP_SWIZZLE_64B))
+                   kQPlanes * ROLAQ_D_C, ROLAQ_D_C * 2, kQK, kQN, CU_TENSOR_MAP_SWIZZLE_64B))
         return ROLAQ_ECUDA;
 
     QuantArgs a;
@@ -246,15 +271,18 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
     a.batch = batch;
     a.heads = heads;
     a.scale_log2 = sm_scale * 1.4426950408889634f;
-    const float lv[4] = {-p->level_b, -p->level_a, p->level_a, p->level_b};
+    uint16_t abits = 0, bbits = 0;
+    float kappa = 1.f;
+    level_encoding(p->level_a, p->level_b, &abits, &bbits, &kappa);
+    const uint16_t lv[4] = {(uint16_t)(bbits | 0x8000u), (uint16_t)(abits | 0x8000u), abits, bbits};
     uint32_t lo = 0, hi = 0;
     for (int c = 0; c < 4; ++c) {
-        const uint16_t bits = bf16_bits(lv[c]);
-        lo |= (uint32_t)(bits & 0xFFu) << (8 * c);
-        hi |= (uint32_t)(bits >> 8) << (8 * c);
+        lo |= (uint32_t)(lv[c] & 0xFFu) << (8 * c);
+        hi |= (uint32_t)(lv[c] >> 8) << (8 * c);
     }
     a.lut_lo = lo;
     a.lut_hi = hi;
+    a.kappa = kappa;
     a.target_items = target;
     a.ws_o = reinterpret_cast<float*>(workspace_dev);
     a.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace_dev) +

@@ -21,7 +21,7 @@ D_R = 64
 PAGE_TOKENS = 64
 PAGE_BYTES = 18432
 TOKEN_BYTES = 288
-RSPLIT_BYTES = 2 * 512 * 512 * 2
+RSPLIT_BYTES = 3 * 512 * 512 * 2
 
 STATUS_BAD_PAGE = 1
 STATUS_BAD_SLOT = 2
@@ -137,10 +137,10 @@ def layer_params_init(tau: float, gain: float) -> rolaq_layer_params:
 
 
 def prepare_rotation(R: torch.Tensor, R_split: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """R: fp32 [512, 512] CUDA (y = c @ R).  Returns the bf16 operand [2, 512, 512]."""
+    """R: fp32 [512, 512] CUDA (y = c @ R).  Returns the bf16 operand [3, 512, 512]."""
     assert R.dtype == torch.float32 and tuple(R.shape) == (D_C, D_C)
     if R_split is None:
-        R_split = torch.empty((2, D_C, D_C), dtype=torch.bfloat16, device=R.device)
+        R_split = torch.empty((3, D_C, D_C), dtype=torch.bfloat16, device=R.device)
     _check("rolaq_prepare_rotation", lib().rolaq_prepare_rotation(_ptr(R), _ptr(R_split), _stream(stream)))
     return R_split
 

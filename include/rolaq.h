@@ -75,8 +75,8 @@ extern "C" {
 #define ROLAQ_PAGE_META_OFFSET  8192
 #define ROLAQ_PAGE_KR_OFFSET    10240
 
-/* Rotation operand prepared by rolaq_prepare_rotation: two bf16 planes [2][512][512]. */
-#define ROLAQ_RSPLIT_BYTES (2u * 512u * 512u * 2u)
+/* Rotation operand prepared by rolaq_prepare_rotation: three bf16 planes [3][512][512]. */
+#define ROLAQ_RSPLIT_BYTES (3u * 512u * 512u * 2u)
 
 /* ---- error codes ---------------------------------------------------------------- */
 #define ROLAQ_OK            0
@@ -126,9 +126,9 @@ int rolaq_layer_params_init(rolaq_layer_params* p, float tau, float gain);
 
 /* Convert the fp32 rotation R_dev [512][512] (row-major, y = c . R for a row vector c)
  * into the tensor-core operand R_split_dev (ROLAQ_RSPLIT_BYTES, 16-B aligned): plane 0
- * holds bf16(R^T), plane 1 holds bf16(R^T - plane0), both [512 out][512 in].  The pair
- * reproduces R to about 2^-17 relative, so y keeps fp32-level accuracy.  Run once per
- * layer at load time.  [S3.3]                                                         */
+ * holds bf16(R^T), plane 1 the nearest bf16 of R^T - plane0, plane 2 the nearest bf16 of
+ * what is left, each [512 out][512 in].  The three planes reproduce R to about 2^-26
+ * relative, so y keeps fp32-level accuracy.  Run once per layer at load time.  [S3.3]                                                         */
 int rolaq_prepare_rotation(const float* R_dev, void* R_split_dev, void* stream);
 
 /* Write path [S3.2], [S3.3], [A.3]: for each of n tokens i, rotate c_dev[i] (bf16 [n][512])

@@ -78,10 +78,11 @@ def _check_write(cache, cs, krs, Rm, pt, seq_lens, tau, gain, n_sink=0, n_recent
                     slot = n_sink + p % n_recent
                 else:
                     continue
-                # bf16 of an fp32 y that is within ~1e-6 relative of the fp64 y: at most
-                # one bf16 ulp apart
+                # bf16 of an fp32 y whose error is ~1e-6 of the token's magnitude: one bf16
+                # ulp apart, plus that error for coordinates near zero
                 d = np.abs(prot[r, slot] - yb[p])
-                assert (d <= np.abs(yb[p]) * 2.0 ** -7 + 1e-30).all()
+                tol = np.abs(yb[p]) * 2.0 ** -7 + 1e-5 * np.abs(q["y"][p]).max()
+                assert (d <= tol).all(), (p, float((d - tol).max()))
     return frac_total / max(n_total, 1)
 
 
@@ -215,3 +216,19 @@ def test_bad_page_entry_sets_status_and_skips():
     xq = O.dequantize(d["q"]["packed"], d["q"]["meta"], 0.9)[keep]
     o_ref, _ = O.attend(f64(q_c[0]), f64(q_r[0]), xq, d["k_r"][keep], SM_SCALE)
     assert rel_l2(out[0].cpu().numpy().astype(np.float64), o_ref).max() <= DECODE_TOL
+
+
+def test_quantize_metadata_tail_over_a_million_groups():
+    """Codes and metadata over 262,144 tokens (1,048,576 groups), the decode-shaped latent
+    distribution: the worst group still meets the tolerances."""
+    w = W.Workload("tail", 1, (262144,), 16, seed=97)
+    tau, gain = 0.93, 1.14
+    cache, cs, krs, Rm, pt = _quantize_on_gpu(w, 0, [262144], tau, gain)
+    packed, meta, kr = O.pages_read_fast(cache.pages.cpu().numpy(), pt, 0, 262144)
+    q = O.quantize(f64(cs[0]), Rm, tau, gain)
+    ok, frac, nbad = codes_match(packed, q, tau)
+    emu, es = meta_match(meta, q, gain)
+    print(f"\nwrite-path tail: codes in window {frac:.2e}, mismatches outside {nbad}, "
+          f"max mean err {emu:.3e}, max scale err {es:.3e}")
+    assert ok, nbad
+    assert emu <= META_TOL and es <= META_TOL, (emu, es)
