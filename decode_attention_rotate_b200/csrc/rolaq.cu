@@ -301,6 +301,46 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
     return launch_status();
 }
 
+// ---- decode with library-owned scratch -------------------------------------------
+// Some callers cannot allocate device memory (a pool or captured allocator owns it, or a
+// host forbids allocation after start-up), so this entry point takes the split-K scratch
+// from a fixed array in the library.  The array is shared by every call on a device and
+// keeps the previous call's contents; the decode kernels write every partial before the
+// merge reads it, so nothing has to be cleared.  Overlapping calls race on it.
+static __device__ __align__(256) unsigned char g_decode_scratch[ROLAQ_STATIC_SCRATCH_BYTES];
+
+namespace {
+// Device address of g_decode_scratch, looked up once per device with that device current
+// (the host-side symbol is only a stand-in and must never reach a kernel).
+void* static_scratch_ptr(int dev) {
+    static void* ptrs[kMaxDevices] = {nullptr};
+    static std::mutex mu;
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return nullptr;
+        ptrs[dev] = p;
+    }
+    return ptrs[dev];
+}
+}  // namespace
+
+int rolaq_decode_attn_static(const rolaq_cache* cache, const rolaq_layer_params* p,
+                             const void* q_c_rot_dev, const void* q_R_dev,
+                             const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
+                             float* out_dev, float* lse_dev, void* stream) {
+    if (heads <= 0 || heads % 16) return ROLAQ_EUNSUPPORTED;
+    if (batch <= 0) return ROLAQ_EINVAL;
+    if (decode_ws_bytes(batch, heads) > (size_t)ROLAQ_STATIC_SCRATCH_BYTES) return ROLAQ_ENOSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ROLAQ_ECUDA;
+    void* scratch = static_scratch_ptr(dev);
+    if (!scratch) return ROLAQ_ECUDA;
+    return rolaq_decode_attn(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale,
+                             out_dev, lse_dev, scratch, (size_t)ROLAQ_STATIC_SCRATCH_BYTES, stream);
+}
+
 int rolaq_get_status(int* bits, void* stream) {
     if (!bits) return ROLAQ_EINVAL;
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return ROLAQ_ECUDA;

@@ -87,6 +87,9 @@ def lib() -> ctypes.CDLL:
         L.rolaq_decode_attn.restype = i32
         L.rolaq_decode_attn.argtypes = [P(rolaq_cache), P(rolaq_layer_params), vp, vp, vp, i32, i32,
                                         ctypes.c_float, vp, vp, vp, sz, vp]
+        L.rolaq_decode_attn_static.restype = i32
+        L.rolaq_decode_attn_static.argtypes = [P(rolaq_cache), P(rolaq_layer_params), vp, vp, vp, i32, i32,
+                                               ctypes.c_float, vp, vp, vp]
         L.rolaq_get_status.restype = i32
         L.rolaq_get_status.argtypes = [P(ctypes.c_int), vp]
         _LIB = L
@@ -207,6 +210,29 @@ def decode_attn(cache: PagedCache, params: rolaq_layer_params, q_c_rot: torch.Te
     _check("rolaq_decode_attn", lib().rolaq_decode_attn(
         ctypes.byref(d), ctypes.byref(params), _ptr(q_c_rot), _ptr(q_r), _ptr(seq_lens), B, H,
         float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+STATIC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def decode_attn_static(cache: PagedCache, params: rolaq_layer_params, q_c_rot: torch.Tensor,
+                       q_r: torch.Tensor, seq_lens: torch.Tensor, sm_scale: float,
+                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       stream=None):
+    """rolaq_decode_attn_static: decode with the library's own scratch array, for callers
+    that cannot allocate device memory.  out / lse must be passed by such callers (the
+    defaults here allocate them for convenience)."""
+    B, H = int(q_c_rot.shape[0]), int(q_c_rot.shape[1])
+    dev = q_c_rot.device
+    if out is None:
+        out = torch.empty((B, H, D_C), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    d = cache.desc()
+    _check("rolaq_decode_attn_static", lib().rolaq_decode_attn_static(
+        ctypes.byref(d), ctypes.byref(params), _ptr(q_c_rot), _ptr(q_r), _ptr(seq_lens), B, H,
+        float(sm_scale), _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
 
 

@@ -170,6 +170,28 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
                       float* out_dev, float* lse_dev,
                       void* workspace_dev, size_t workspace_bytes, void* stream);
 
+/* Decode without a caller-provided workspace.  Same arguments, result and errors as
+ * rolaq_decode_attn, except that the split-K scratch lives in a fixed array inside the
+ * library (ROLAQ_STATIC_SCRATCH_BYTES per GPU, held by every GPU that loads the library
+ * until the process exits) instead of caller memory.  It is for callers that cannot call
+ * cudaMalloc: code running while a memory pool or a captured allocator owns the device
+ * memory, plug-ins that are handed tensors but no allocator, and hosts that forbid
+ * allocation after start-up.  The call itself allocates nothing.
+ *   - The first call on each device looks up the array's device address on that device;
+ *     make that first call before any stream capture.
+ *   - Requests whose scratch would exceed ROLAQ_STATIC_SCRATCH_BYTES (that is,
+ *     rolaq_decode_workspace_bytes(batch, heads) > ROLAQ_STATIC_SCRATCH_BYTES) return
+ *     ROLAQ_ENOSPACE before anything is launched.
+ *   - Every call on a device shares the one array and leaves its contents behind; the
+ *     kernels overwrite whatever they read, so nothing needs clearing, but calls that can
+ *     overlap on the GPU (different streams without ordering between them) race on it.
+ * The paper has no counterpart of this entry point; it is an integration convenience.   */
+#define ROLAQ_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int rolaq_decode_attn_static(const rolaq_cache* cache, const rolaq_layer_params* p,
+                             const void* q_c_rot_dev, const void* q_R_dev,
+                             const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
+                             float* out_dev, float* lse_dev, void* stream);
+
 /* Copy the device status word of the current device to *bits and clear it.  Blocks until
  * `stream` has finished.                                                              */
 int rolaq_get_status(int* bits, void* stream);
