@@ -33,9 +33,11 @@ METRIC = "2-bit MLA decode: cache GB/s & % HBM roofline; quantize-append tokens/
 SM_SCALE = 1.0 / math.sqrt(192.0)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-# DRAM bytes (read + write) per launch of the decode split kernel from the committed ncu
-# capture (profiles/); None until a capture of the current kernel exists.
-DECODE_TRAFFIC_PER_LAUNCH = None
+# DRAM bytes (read + write) per decode launch of the bench workload, from the ncu capture
+# summarised in profiles/decode_split_4x128k_h16.md (4 x 131,072 tokens): reads 151.18 MB
+# scale with the tokens (x2 here), the 5.79 MB of split-K partials depend only on the item
+# count, which is the same; None whenever the kernel has changed since that capture.
+DECODE_TRAFFIC_PER_LAUNCH = 2 * 151.18e6 + 5.79e6
 
 
 def peaks():
@@ -65,7 +67,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -228,7 +230,6 @@ def run_ours(args, rank, world, dev):
     t1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    clocks = sampler.stop()
     total_ms = t0.elapsed_time(t1)
     # decode-call durations: the last step's events (all steps are identical launches)
     dec_ms = sum(ev[l][0].elapsed_time(ev[l][1]) for l in range(w.layers)) / w.layers
@@ -274,6 +275,7 @@ def run_ours(args, rank, world, dev):
 
     # prefill write path: 65,536 tokens x 27 layers
     q_stats = bench_quantize(args, dev, world)
+    clocks = sampler.stop()     # sampled across the three timed regions
 
     hbm, bf16, src = peaks()
     dec_bytes = w.total_tokens * R.TOKEN_BYTES
@@ -345,9 +347,51 @@ def bench_quantize(args, dev, world):
             "roofline": {"bound": "tensor", "achieved": round(flops / (per_launch_ms * 1e-3) / 1e12, 1),
                          "peak": bf16, "unit": "TFLOP/s",
                          "frac": round(flops / (per_launch_ms * 1e-3) / 1e12 / bf16, 4),
-                         "executed_flops_factor": 2, "peak_source": src},
+                         "executed_flops_factor": 3, "peak_source": src},
             "hbm": {"achieved": round(bytes_ / (per_launch_ms * 1e-3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
                     "frac": round(bytes_ / (per_launch_ms * 1e-3) / 1e9 / hbm, 4)}}
+
+
+# ------------------------------------------------------------ profiling cases ----
+# Small single-kernel cases for ncu captures (inputs larger than L2, a few hundred MB on
+# the device): `--case decode` runs one layer of 4 requests x 131,072 tokens at 16 heads,
+# `--case quantize` the write path on 262,144 tokens.  They print their own timing.
+
+def run_case(args, dev):
+    if args.case == "decode":
+        w = W.Workload("decode_4x128k_h16", 4, (131072,) * 4, 16, seed=4242)
+        lay = DecodeLayer(w, 0, dev)
+        lay.fill(w, 0, dev)
+        ws = torch.empty(R.decode_workspace_bytes(w.batch, w.heads), dtype=torch.uint8, device=dev)
+        lens = torch.as_tensor(w.seq_lens, dtype=torch.int32, device=dev)
+        fn = lambda: R.decode_attn(lay.cache, lay.params, lay.q_c, lay.q_r, lens, SM_SCALE, lay.out, lay.lse, ws)
+        nbytes = w.total_tokens * R.TOKEN_BYTES
+    else:
+        w = W.Workload("quantize_262k", 1, (262144,), 16, seed=4243)
+        n = w.total_tokens
+        tau, gain = W.layer_constants(w, 0)
+        pt = torch.as_tensor(W.page_table(w))
+        cache = R.PagedCache(int(pt.max()) + 1, pt, device=dev)
+        Rs = R.prepare_rotation(torch.as_tensor(W.rotation(w.seed)).to(dev))
+        p = R.layer_params_init(tau, gain)
+        c = W.latent_device(w, 0, n, dev)
+        kr = W.rope_key_device(w, 0, n, dev)
+        req = torch.zeros(n, dtype=torch.int32, device=dev)
+        pos = torch.arange(n, dtype=torch.int32, device=dev)
+        fn = lambda: R.quantize_append(cache, p, Rs, c, kr, req, pos)
+        nbytes = n * (1024 + 128 + 288)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"case": args.case, "workload": w.name, "ms_per_call": round(ms, 4),
+                      "algorithmic_GBps": round(nbytes / ms / 1e6, 1), "status": R.get_status()}), flush=True)
 
 
 # ---------------------------------------------------------------- reference arm ----
@@ -412,6 +456,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["decode", "quantize"], default=None,
+                    help="run one small single-kernel case (for ncu captures) instead of the bench")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 1)
 
@@ -428,6 +474,9 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     R.lib()
+    if args.case:
+        run_case(args, dev)
+        return
     res = run_ours(args, rank, world, dev)
     if rank == 0:
         print(json.dumps(res), flush=True)

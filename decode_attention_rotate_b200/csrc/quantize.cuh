@@ -371,3 +371,133 @@ __global__ void rolaq_split_rotation(const float* __restrict__ R, __nv_bfloat16*
 }
 
 }  // namespace rolaq
+
+namespace rolaq {
+
+// ---- small appends --------------------------------------------------------------
+// A decode step appends one token per request: a few tokens per call.  The tensor-core
+// kernel above would stream all of R through a single CTA for them, so small calls use
+// this kernel instead: one CTA of 16 warps per (group, 8 tokens).  Warp w computes output
+// coordinates 128g + 8w .. +7: for each, the 32 lanes read the three R-plane rows
+// coalesced (16 inputs each), sum the planes in fp32 (smallest first), multiply-add the
+// CTA's tokens and reduce across the warp.  The group statistics are block reductions.
+constexpr int kSmallTok = 8;
+constexpr int kSmallMaxN = 64;
+constexpr int kSmallThreads = 512;
+constexpr int kSmallOutPerWarp = ROLAQ_GROUP / (kSmallThreads / 32);   // 8
+
+__device__ __forceinline__ float block_sum128(float v, float* red) {
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const float r = (red[0] + red[1]) + (red[2] + red[3]);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    return r;
+}
+
+__global__ void __launch_bounds__(kSmallThreads)
+rolaq_quantize_small_kernel(const __nv_bfloat16* __restrict__ R_split, const __nv_bfloat16* __restrict__ c,
+                            const QuantArgs args) {
+    __shared__ __align__(16) __nv_bfloat16 s_c[kSmallTok][ROLAQ_D_C];
+    __shared__ float s_y[kSmallTok][ROLAQ_GROUP];
+    __shared__ float s_red[4];
+    __shared__ uint32_t s_codes[kSmallTok][8];
+    const int g = blockIdx.x;                    // group
+    const int t0 = blockIdx.y * kSmallTok;
+    const int nt = min(kSmallTok, args.n - t0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = threadIdx.x; e < kSmallTok * ROLAQ_D_C / 8; e += blockDim.x) {
+        const int t = e / (ROLAQ_D_C / 8), k8 = e % (ROLAQ_D_C / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (t < nt) v = reinterpret_cast<const uint4*>(c + (size_t)(t0 + t) * ROLAQ_D_C)[k8];
+        reinterpret_cast<uint4*>(s_c[t])[k8] = v;
+    }
+    if (threadIdx.x < kSmallTok * 8) s_codes[threadIdx.x >> 3][threadIdx.x & 7] = 0;
+    __syncthreads();
+    // this lane's 16 inputs of every token, as fp32
+    const size_t plane = (size_t)ROLAQ_D_C * ROLAQ_D_C;
+#pragma unroll 2
+    for (int oo = 0; oo < kSmallOutPerWarp; ++oo) {
+        const int o = kSmallOutPerWarp * warp + oo;
+        float rk[16];
+#pragma unroll
+        for (int q8 = 0; q8 < 16; ++q8) rk[q8] = 0.f;
+#pragma unroll
+        for (int pl = 2; pl >= 0; --pl) {        // smallest plane first
+            const uint4* row = reinterpret_cast<const uint4*>(R_split + pl * plane + (size_t)(128 * g + o) * ROLAQ_D_C);
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {
+                const uint4 u = row[2 * lane + hv];
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    rk[8 * hv + 2 * q] += __uint_as_float(w[q] << 16);
+                    rk[8 * hv + 2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+                }
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < kSmallTok; ++t) {
+            float acc = 0.f;
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {
+                const uint4 cu = reinterpret_cast<const uint4*>(s_c[t])[2 * lane + hv];
+                const uint32_t cw[4] = {cu.x, cu.y, cu.z, cu.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc = fmaf(__uint_as_float(cw[q] << 16), rk[8 * hv + 2 * q], acc);
+                    acc = fmaf(__uint_as_float(cw[q] & 0xFFFF0000u), rk[8 * hv + 2 * q + 1], acc);
+                }
+            }
+            for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (lane == 0) s_y[t][o] = acc;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x >= ROLAQ_GROUP) return;      // warps 0..3 finish the group
+    const int j = threadIdx.x;
+    for (int t = 0; t < nt; ++t) {
+        const int tok = t0 + t;
+        const float y = s_y[t][j];
+        const float mean = block_sum128(y, s_red) * (1.f / 128.f);
+        const float d = y - mean;
+        const float sd = sqrtf(block_sum128(d * d, s_red) * (1.f / 128.f));
+        const float inv = sd > 0.f ? 1.f / sd : 0.f;
+        const float z = d * inv;
+        const uint32_t code = (uint32_t)(z >= -args.tau) + (uint32_t)(z >= 0.f) + (uint32_t)(z >= args.tau);
+        atomicOr(&s_codes[t][j >> 4], code << (2 * (j & 15)));
+        const int rq = args.req[tok], ps = args.pos[tok];
+        long long pid = -1;
+        if (rq >= 0 && rq < args.batch && ps >= 0 && (ps / ROLAQ_PAGE_TOKENS) < args.max_pages) {
+            pid = args.page_table[(long long)rq * args.max_pages + ps / ROLAQ_PAGE_TOKENS];
+            if (pid >= args.num_pages) pid = -1;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (pid < 0) {
+            if (j == 0 && g == 0) raise_status(ROLAQ_STATUS_BAD_SLOT);
+            continue;
+        }
+        uint8_t* page = args.pages + pid * (long long)ROLAQ_PAGE_BYTES;
+        const int row = ps % ROLAQ_PAGE_TOKENS;
+        if (j < 8)
+            reinterpret_cast<uint32_t*>(page + ROLAQ_PAGE_CODES_OFFSET + row * ROLAQ_CODE_BYTES + 32 * g)[j] = s_codes[t][j];
+        if (j == 0)
+            *reinterpret_cast<float2*>(page + ROLAQ_PAGE_META_OFFSET + row * ROLAQ_META_BYTES + 8 * g) =
+                make_float2(mean, args.gain * sd);
+        if (g == 0 && j < 16)
+            reinterpret_cast<uint2*>(page + ROLAQ_PAGE_KR_OFFSET + row * ROLAQ_KR_BYTES)[j] =
+                reinterpret_cast<const uint2*>(args.k_r + (size_t)tok * ROLAQ_D_R)[j];
+        if (args.prot) {
+            const int nslot = args.n_sink + args.n_recent;
+            long long prow = -1;
+            if (ps < args.n_sink)
+                prow = (long long)rq * nslot + ps;
+            else if (args.n_recent > 0 && ps >= args.seq_lens[rq] - args.n_recent)
+                prow = (long long)rq * nslot + args.n_sink + ps % args.n_recent;
+            if (prow >= 0) args.prot[prow * ROLAQ_D_C + 128 * g + j] = __float2bfloat16_rn(y);
+        }
+    }
+}
+
+}  // namespace rolaq

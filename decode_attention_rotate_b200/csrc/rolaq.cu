@@ -190,6 +190,29 @@ int rolaq_quantize_append(const rolaq_cache* cache, const rolaq_layer_params* p,
         return ROLAQ_EINVAL;
     if (cache->n_recent > 0 && !seq_lens_dev) return ROLAQ_EINVAL;
 
+    if (n <= kSmallMaxN) {
+        QuantArgs a;
+        a.pages = reinterpret_cast<uint8_t*>(cache->pages_dev);
+        a.num_pages = cache->num_pages;
+        a.page_table = cache->page_table_dev;
+        a.max_pages = cache->max_pages_per_seq;
+        a.batch = cache->batch;
+        a.prot = (cache->n_sink + cache->n_recent > 0) ? reinterpret_cast<__nv_bfloat16*>(cache->prot_dev) : nullptr;
+        a.n_sink = cache->n_sink;
+        a.n_recent = cache->n_recent;
+        a.req = req_dev;
+        a.pos = pos_dev;
+        a.seq_lens = seq_lens_dev;
+        a.k_r = reinterpret_cast<const __nv_bfloat16*>(k_R_dev);
+        a.n = n;
+        a.tau = p->tau;
+        a.gain = p->gain;
+        dim3 grid(ROLAQ_GROUPS, (n + kSmallTok - 1) / kSmallTok);
+        rolaq_quantize_small_kernel<<<grid, kSmallThreads, 0, (cudaStream_t)stream>>>(
+            reinterpret_cast<const __nv_bfloat16*>(R_split_dev), reinterpret_cast<const __nv_bfloat16*>(c_dev), a);
+        return launch_status();
+    }
+
     CUtensorMap map_c, map_r;
     if (!encode_2d(&map_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(c_dev), ROLAQ_D_C,
                    (uint64_t)n, ROLAQ_D_C * 2, kQK, kQTileM, CU_TENSOR_MAP_SWIZZLE_64B) ||
@@ -296,7 +319,7 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
     cudaStream_t s = (cudaStream_t)stream;
     rolaq_decode_split<<<dim3(items_cap, heads / 16), kDecodeThreads, smem, s>>>(map32, map8, a);
     if ((rc = launch_status())) return rc;
-    rolaq_decode_merge<<<dim3(batch, heads), 128, 0, s>>>(a.ws_o, a.ws_ml, seq_lens_dev, batch, heads,
+    rolaq_decode_merge<<<dim3(batch, heads), kMergeThreads, 0, s>>>(a.ws_o, a.ws_ml, seq_lens_dev, batch, heads,
                                                          target, out_dev, lse_dev);
     return launch_status();
 }

@@ -232,3 +232,68 @@ def test_quantize_metadata_tail_over_a_million_groups():
           f"max mean err {emu:.3e}, max scale err {es:.3e}")
     assert ok, nbad
     assert emu <= META_TOL and es <= META_TOL, (emu, es)
+
+
+def test_streaming_append_with_recent_ring():
+    """Prefill, then one token per request per step (the small-append kernel), with 4 sink
+    and 16 recent tokens protected: every record, the side store after the ring has
+    wrapped, and the decode of the final cache match the oracle."""
+    L0 = [100, 64, 130]
+    steps = 20
+    B = len(L0)
+    tau, gain = 0.94, 1.09
+    n_sink, n_recent = 4, 16
+    w = W.Workload("stream", B, tuple(l + steps for l in L0), 16, paged_shuffled=True, seed=98)
+    Rm = W.rotation(w.seed)
+    R_split = R.prepare_rotation(torch.as_tensor(Rm).to(DEV))
+    pt = W.page_table(w)
+    cache = R.PagedCache(int(pt.max() + 1), torch.as_tensor(pt), n_sink, n_recent, device=DEV)
+    p = R.layer_params_init(tau, gain)
+    Lf = [l + steps for l in L0]
+    lat = [W.latent(w, 0, Lf[r], stream=100 + r) for r in range(B)]
+    kr = [W.rope_key(w, 0, Lf[r], stream=200 + r) for r in range(B)]
+    # prefill (tensor-core path for the 294 tokens)
+    c = torch.cat([lat[r][:L0[r]] for r in range(B)]).to(DEV)
+    k = torch.cat([kr[r][:L0[r]] for r in range(B)]).to(DEV)
+    req = torch.cat([torch.full((L0[r],), r, dtype=torch.int32) for r in range(B)]).to(DEV)
+    pos = torch.cat([torch.arange(L0[r], dtype=torch.int32) for r in range(B)]).to(DEV)
+    R.quantize_append(cache, p, R_split, c, k, req, pos, torch.as_tensor(L0, dtype=torch.int32).to(DEV))
+    # one token per request per step
+    for s in range(steps):
+        c = torch.stack([lat[r][L0[r] + s] for r in range(B)]).to(DEV)
+        k = torch.stack([kr[r][L0[r] + s] for r in range(B)]).to(DEV)
+        req = torch.arange(B, dtype=torch.int32, device=DEV)
+        pos = torch.as_tensor([L0[r] + s for r in range(B)], dtype=torch.int32).to(DEV)
+        lens = torch.as_tensor([L0[r] + s + 1 for r in range(B)], dtype=torch.int32).to(DEV)
+        R.quantize_append(cache, p, R_split, c, k, req, pos, lens)
+    torch.cuda.synchronize()
+    pool = cache.pages.cpu().numpy()
+    prot = cache.prot.float().cpu().numpy().astype(np.float64)
+    q_c, q_r = W.queries(w, 0)
+    lens = torch.as_tensor(Lf, dtype=torch.int32).to(DEV)
+    out, _ = R.decode_attn(cache, p, q_c.to(DEV), q_r.to(DEV), lens, SM_SCALE)
+    out = out.cpu().numpy().astype(np.float64)
+    for r in range(B):
+        L = Lf[r]
+        q = O.quantize(f64(lat[r]), Rm.astype(np.float64), tau, gain)
+        packed, meta, krb = O.pages_read_fast(pool, pt, r, L)
+        ok, frac, nbad = codes_match(packed, q, tau)
+        assert ok, (r, nbad)
+        emu, es = meta_match(meta, q, gain)
+        assert emu <= META_TOL and es <= META_TOL, (r, emu, es)
+        assert (krb == bf16_bits(kr[r])).all()
+        yb = O.bf16_round(q["y"])
+        content = np.zeros((L, 512))
+        for pp in range(L):
+            if pp < n_sink:
+                slot = pp
+            elif pp >= L - n_recent:
+                slot = n_sink + pp % n_recent
+            else:
+                continue
+            d = np.abs(prot[r, slot] - yb[pp])
+            assert (d <= np.abs(yb[pp]) * 2.0 ** -7 + 1e-5 * np.abs(q["y"][pp]).max()).all(), (r, pp)
+            content[pp] = prot[r, slot]
+        o_ref, _ = O.decode_request(f64(q_c[r]), f64(q_r[r]), packed, meta, O.bf16_bits_to_f64(krb), tau,
+                                    SM_SCALE, content, n_sink, n_recent)
+        assert rel_l2(out[r], o_ref).max() <= DECODE_TOL
