@@ -37,7 +37,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # summarised in profiles/decode_split_4x128k_h16.md (4 x 131,072 tokens): reads 151.18 MB
 # scale with the tokens (x2 here), the 5.79 MB of split-K partials depend only on the item
 # count, which is the same; None whenever the kernel has changed since that capture.
-DECODE_TRAFFIC_PER_LAUNCH = 2 * 151.18e6 + 5.79e6
+DECODE_TRAFFIC_PER_LAUNCH = None
 
 
 def peaks():

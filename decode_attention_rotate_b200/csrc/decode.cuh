@@ -3,25 +3,31 @@
 // softmax over the request's tokens, 512-d latent readout in the rotated basis.
 //
 // Kernel A (rolaq_decode_split): one CTA per (work item, 16-head chunk).  A work item is a
-// run of whole pages of one request (split-K over the sequence).  8 warps in two teams of
-// four.  Team t owns tokens 32t..32t+31 of every page: lane 0 of its warp 0 issues the
-// bulk tensor copies of that half page (codes, metadata, RoPE rows; 128-byte swizzle)
-// into the team's ring of shared-memory stages, and the team keeps its own online-softmax
-// state.  Inside a team, warp g owns content-channel group g (128 channels) and RoPE
-// channels 16g..16g+15.
+// run of whole pages of one request (split-K over the sequence).  16 warps in four teams
+// of four; team t takes pages t, t+4, t+8, ... of the item and keeps its own online
+// softmax state, and the four teams are merged inside the CTA at the end, so each item
+// writes one partial.  Lane 0 of a team's first warp streams its pages (one 144-row bulk
+// tensor copy per page, 128-byte swizzle) through two shared-memory stages and issues the
+// team's tensor-core MMAs.  Inside a team, warp q owns content channels 32q..32q+31 of
+// every 128-channel group (the TMEM lane quarter it may access) and RoPE channels
+// 16q..16q+15.
 //
-// A team walks its tokens in steps of 16 as a software pipeline with one team barrier per
-// step: QK(j+1) | barrier | softmax(j+1) and PV(j).
-//   QK    mma.sync m16n8k16 (heads = M) on bf16 level fragments built in registers from
-//         the codes (PRMT lookup); the group metadata is folded outside the MMA
-//         (q.x = mean * sum(q_g) + scale * (q_g . level)); partial scores per group go to
-//         shared memory.
-//   softmax  warp g sums the four partials for heads 4g..4g+3; the running max moves only
-//         when a score exceeds it by more than 2^8 (checked with one warp vote), so the
-//         common step has no shuffles; row sums stay per lane until the end.
-//   PV    the same level fragments transposed in registers (movmatrix), the scale folded
-//         into P, the mean term kept as a per-head rank-1 accumulator.
-// Kernel B (rolaq_decode_merge): log-sum-exp merge of the per-(item, team) partials.
+// A team walks its tokens in steps of 16 with one team barrier per step:
+//   dequant  per (token, group) the four fp16 values mean + scale * level are prepared
+//            one step ahead; a PRMT lookup turns every 2-bit code straight into x (fp16;
+//            bf16 would round all channels sharing a code the same way and cost ~5x in
+//            output error).
+//   QK       mma.sync m16n8k16 (heads = M) on those x fragments in registers; partial
+//            scores of the four warps meet in shared memory.
+//   A tile   the same fragments transposed (movmatrix) and stored to tensor memory with
+//            lanes = channels, columns = tokens (two-slot ring).
+//   softmax  warp q takes heads 4q..4q+3; the running max moves only when a score exceeds
+//            it by more than 2^8 (one warp vote in the common case); probabilities go to
+//            shared memory as the fp16 B operand.
+//   PV       tcgen05.mma M = 128 channels of a group, N = 16 heads, K = 16 tokens, A from
+//            tensor memory, accumulating O (fp32) in tensor memory; a rare rescale pass
+//            multiplies O when a head's running max moves.
+// Kernel B (rolaq_decode_merge): log-sum-exp merge of the per-item partials.
 #pragma once
 #include "common.cuh"
 
@@ -29,15 +35,18 @@ namespace rolaq {
 
 constexpr int kPageTok = ROLAQ_PAGE_TOKENS;
 constexpr int kPageRows = ROLAQ_PAGE_BYTES / 128;   // 144 rows of 128 B
-constexpr int kNStage = 8;                          // half-page stages per team
-constexpr int kStepTok = 16;                        // tokens per pipeline step
-constexpr int kSStride = 24;                        // floats per head row of sT / sP
-constexpr int kDecodeThreads = 256;
+constexpr int kTeams = 4;
+constexpr int kDecodeThreads = 128 * kTeams;
+constexpr int kStages = 2;                          // whole pages in flight per team
+constexpr int kRing = 2;                            // TMEM A slots / P tiles per team
+constexpr int kStepTok = 16;                        // tokens per step
+constexpr int kRingCol = 64;                        // O: columns 0..63 (16 per group)
+constexpr int kTeamCols = kRingCol + 32 * kRing;    // TMEM columns per team (ring after O)
+static_assert(kTeams * kTeamCols <= 512, "tensor memory columns");
+constexpr int kLutStride = 6;                       // uint2 per token row of the LUT tile
 constexpr float kRescaleLog2 = 8.f;
-// A team stages its half of a page: 32 code rows, 8 metadata rows, 32 RoPE rows.
-constexpr int kHalfBytes = 9216;
-constexpr int kHalfMetaOff = 4096;                  // smem row 32
-constexpr int kHalfKrOff = 5120;                    // smem row 40
+constexpr int kMetaRow = 64;                        // page rows: codes 0..63, meta 64..79,
+constexpr int kKrRow = 80;                          // RoPE keys 80..143
 
 struct DecodeArgs {
     const int32_t* page_table;
@@ -50,23 +59,28 @@ struct DecodeArgs {
     const int32_t* seq_lens;
     int batch, heads;
     float scale_log2;            // sm_scale * log2(e)
-    uint32_t lut_lo, lut_hi;     // low / high bytes of the four bf16 levels / kappa
-    float kappa;                 // level = kappa * bf16 level
+    float level_a, level_b;      // reconstruction levels (fp32)
     int target_items;
-    float* ws_o;                 // [items][2][heads][512]
-    float2* ws_ml;               // [items][2][heads]  (reference max (log2 units), sum)
+    float* ws_o;                 // [items][heads][512]  sum_t 2^(s_t - m) x_t
+    float2* ws_ml;               // [items][heads]       (m (log2 units), sum_t 2^(s_t - m))
 };
 
 struct DecodeSmem {
-    alignas(1024) uint8_t stage[2][kNStage][kHalfBytes];
-    float sT[2][2][4][16][kSStride];     // [team][buffer][group][head][token]
-    float sP[2][2][16][kSStride];        // [team][buffer][head][token]
-    float sAl[2][2][16];                 // [team][buffer][head] rescale factor
-    alignas(8) uint64_t full[2][kNStage];
-    int valid[2][kNStage];
+    alignas(1024) uint8_t stage[kTeams][kStages][ROLAQ_PAGE_BYTES];
+    float sT[kTeams][2][4][16][16];          // partial scores [team][buf][warp][head][token']
+    alignas(128) uint8_t P[kTeams][kRing][512];   // fp16 probabilities, UMMA B layout
+    alignas(16) uint2 lut[kTeams][2][kStepTok][kLutStride];   // (lo, hi) bytes of 4 x values
+    float sAl[kTeams][2][16];                // rescale factor per head
+    float2 team_ml[kTeams][16];
+    int resc[kTeams][2];
+    alignas(8) uint64_t full[kTeams][kStages];
+    alignas(8) uint64_t pvbar[kTeams][kRing];
+    int valid[kTeams][kStages];
+    uint32_t tmem_base;
     int plan[4];
     int abort;
 };
+static_assert(sizeof(DecodeSmem) + 1024 <= 227 * 1024, "decode shared memory");
 
 // ---- split plan --------------------------------------------------------------
 // pages_b = ceil(L_b / 64); chunk = max(1, ceil(sum_b pages_b / target)); request b
@@ -132,53 +146,56 @@ __device__ PlanInfo plan_lookup(const int32_t* seq_lens, int batch, int target, 
     return pi;
 }
 
-// Channel (within a 128-channel group) that QK k-slice s, MMA k index kk maps to.
-// Thread i = lane % 4 loads code bytes 8i..8i+7 of the group; its fragment values are
-// channels 32i + 16*(s/4) + 8*(kk/8) + 4*(kk%2) + s%4 (any channel order works for a
-// dot product as long as the query fragments follow it).
-__device__ __forceinline__ int qk_channel(int s, int kk) {
-    return 32 * ((kk & 7) >> 1) + 16 * (s >> 2) + 8 * (kk >> 3) + 4 * (kk & 1) + (s & 3);
+// Instruction descriptor of the PV MMA: f16 x f16 -> f32, M = 128, N = 16.
+constexpr uint32_t kPvIdesc = (1u << 4) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr float kF16Max = 65504.f;
+
+// Shared-memory descriptor of a K-major operand without swizzle: 8-row x 16-byte core
+// matrices, K-adjacent cores 128 B apart, 8-row groups 256 B apart.
+__device__ __forceinline__ uint64_t umma_desc_plain(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 16) |
+           ((uint64_t)(256 >> 4) << 32) | (1ull << 46);
+}
+// D (tensor memory) (+)= A (tensor memory) * B (shared memory)
+__device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t acc) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                 :: "r"(d), "r"(a), "l"(bdesc), "r"(kPvIdesc), "r"(acc) : "memory");
+}
+// Eight fp16 pairs from one 32-bit word of codes: bytes 0-1 hold 8 codes of token A,
+// bytes 2-3 8 codes of token B (code j of a byte at bits 2j).  r[k][0] = (x_A of code k
+// of byte 0, x_A of code k of byte 1); r[k][1] the same for token B.  A token's lookup
+// pair (lo, hi) holds the low and high bytes of its four fp16 x values, so PRMT nibbles
+// c and c + 4 pick value c: the selector of a byte pair is byte * 0x11 + 0x4040 with the
+// code moved to bits 0-1; __umulhi(m, 0x11 << (16 - s)) does the same for bytes 2-3
+// (every multiplier fits in 32 bits).
+__device__ __forceinline__ void dequant_word2(uint32_t w, uint2 la, uint2 lb, uint32_t (&r)[4][2]) {
+    const uint32_t m0 = w & 0x03030303u;
+    r[0][0] = prmt(la.x, la.y, m0 * 0x11u + 0x4040u);
+    r[0][1] = prmt(lb.x, lb.y, __umulhi(m0, 0x11u << 16) + 0x4040u);
+    const uint32_t m1 = w & 0x0C0C0C0Cu;
+    r[1][0] = prmt(la.x, la.y, (m1 >> 2) * 0x11u + 0x4040u);
+    r[1][1] = prmt(lb.x, lb.y, __umulhi(m1, 0x11u << 14) + 0x4040u);
+    const uint32_t m2 = w & 0x30303030u;
+    r[2][0] = prmt(la.x, la.y, (m2 >> 4) * 0x11u + 0x4040u);
+    r[2][1] = prmt(lb.x, lb.y, __umulhi(m2, 0x11u << 12) + 0x4040u);
+    const uint32_t m3 = w & 0xC0C0C0C0u;
+    r[3][0] = prmt(la.x, la.y, __umulhi(m3, 0x11u << 26) + 0x4040u);
+    r[3][1] = prmt(lb.x, lb.y, __umulhi(m3, 0x11u << 10) + 0x4040u);
 }
 
-// Four bf16 level pairs from one 32-bit word of codes (16 codes, 2 bit each).
-// Output r[k][0] = (level(code k), level(code 4+k)), r[k][1] = (code 8+k, code 12+k).
-// Selector byte for code c is c | (c + 4) << 4: PRMT takes the low level byte from
-// lut_lo[c] and the high byte from lut_hi[c].  (m >> 2k) * 0x11 spreads the code in each
-// byte to both nibbles; __umulhi(m, 0x11 << (16 - 2k)) does the same and moves bytes 2..3
-// down to 0..1 (every multiplier must fit in 32 bits).
-__device__ __forceinline__ void dequant_word(uint32_t w, uint32_t lo, uint32_t hi,
-                                             uint32_t (&r)[4][2]) {
-    uint32_t m0 = w & 0x03030303u;
-    r[0][0] = prmt(lo, hi, m0 * 0x11u + 0x40404040u);
-    r[0][1] = prmt(lo, hi, __umulhi(m0, 0x11u << 16) + 0x4040u);
-    uint32_t m1 = w & 0x0C0C0C0Cu;
-    r[1][0] = prmt(lo, hi, (m1 >> 2) * 0x11u + 0x40404040u);
-    r[1][1] = prmt(lo, hi, __umulhi(m1, 0x11u << 14) + 0x4040u);
-    uint32_t m2 = w & 0x30303030u;
-    r[2][0] = prmt(lo, hi, (m2 >> 4) * 0x11u + 0x40404040u);
-    r[2][1] = prmt(lo, hi, __umulhi(m2, 0x11u << 12) + 0x4040u);
-    uint32_t m3 = w & 0xC0C0C0C0u;
-    r[3][0] = prmt(lo, hi, __umulhi(m3, 0x11u << 26) + 0x40404040u);
-    r[3][1] = prmt(lo, hi, __umulhi(m3, 0x11u << 10) + 0x4040u);
-}
-
-// Issue the three copies of one team's half of page `page_idx` into stage k % kNStage
-// (or mark it invalid when the page-table entry is outside the pool).
-__device__ __forceinline__ void load_half_page(DecodeSmem& sm, const CUtensorMap* map32,
-                                               const CUtensorMap* map8, const DecodeArgs& args,
-                                               int team, int b, int page_idx, int k) {
-    const int st = k % kNStage;
+// Issue the bulk copy of one page (all 144 rows) into stage k % kStages, or mark the
+// stage invalid when the page-table entry is outside the pool.
+__device__ __forceinline__ void load_page(DecodeSmem& sm, const CUtensorMap* map, const DecodeArgs& args,
+                                          int team, int b, int page_idx, int k) {
+    const int st = k % kStages;
     long long pid = -1;
     if (page_idx < args.max_pages) pid = args.page_table[(long long)b * args.max_pages + page_idx];
     const uint32_t bar = smem_u32(&sm.full[team][st]);
     if (pid >= 0 && pid < args.num_pages) {
         sm.valid[team][st] = 1;
-        const int row0 = (int)(pid * kPageRows);
-        const uint32_t dst = smem_u32(sm.stage[team][st]);
-        mbar_arrive_expect_tx(bar, kHalfBytes);
-        tma_load_2d(dst, map32, 0, row0 + 32 * team, bar);
-        tma_load_2d(dst + kHalfMetaOff, map8, 0, row0 + 64 + 8 * team, bar);
-        tma_load_2d(dst + kHalfKrOff, map32, 0, row0 + 80 + 32 * team, bar);
+        mbar_arrive_expect_tx(bar, ROLAQ_PAGE_BYTES);
+        tma_load_2d(smem_u32(sm.stage[team][st]), map, 0, (int)(pid * kPageRows), bar);
     } else {
         sm.valid[team][st] = 0;
         raise_status(ROLAQ_STATUS_BAD_PAGE);
@@ -186,121 +203,153 @@ __device__ __forceinline__ void load_half_page(DecodeSmem& sm, const CUtensorMap
     }
 }
 
-// Per-warp state of a team's pipeline.
-struct StepRegs {
-    uint32_t bq[2][8][2];    // level fragments of the step's two n-tiles (8 tokens each)
-    float mu[2][2], sc[2][2];  // mean and kappa*scale of the fragment-column tokens
-};
+// Lookup pair of token tt (0..15 of step `sub` of a staged page), group gg: fp16 of
+// mean + scale * (-b, -a, a, b), split into low bytes and high bytes.  Tokens past the
+// sequence end or on an invalid page get zeros, so their x is 0 (their scores are masked).
+// Values beyond the fp16 range raise ROLAQ_STATUS_RANGE.
+__device__ __forceinline__ void lut_prep(const uint8_t* pg, bool vpage, int sub, int tt, int gg, int pos,
+                                         int L, float la, float lb, uint2* lut) {
+    uint2 v = make_uint2(0u, 0u);
+    if (vpage && pos < L) {
+        const int pt = kStepTok * sub + tt;
+        const float2 ms = *reinterpret_cast<const float2*>(
+            pg + swz128(kMetaRow + (pt >> 2), (pt & 3) * 32 + 8 * gg));
+        if (!(fabsf(ms.x) + fabsf(ms.y) * lb < kF16Max)) raise_status(ROLAQ_STATUS_RANGE);
+        const uint32_t w01 = pack_f16(fmaf(ms.y, -lb, ms.x), fmaf(ms.y, -la, ms.x));
+        const uint32_t w23 = pack_f16(fmaf(ms.y, la, ms.x), fmaf(ms.y, lb, ms.x));
+        v.x = prmt(w01, w23, 0x6420u);
+        v.y = prmt(w01, w23, 0x7531u);
+    }
+    lut[tt * kLutStride + gg] = v;
+}
 
-// QK for one 16-token step (rows 16*sub.. of the staged half page) and this warp's group:
-// dequantise, MMA, fold the metadata, add the RoPE part, store the partial scores.
-// FULL: all 16 tokens are in the sequence and none is protected.
-template <bool FULL>
-__device__ __forceinline__ void qk_step(const uint8_t* pg, int sub, float (*sT)[kSStride], int r, int i,
-                                        int g, uint32_t lut_lo, uint32_t lut_hi, float kappa,
-                                        const uint32_t (&qa)[8][4], const uint32_t (&qra)[4],
-                                        float qs0, float qs1, int nvalid, int pos0, int L,
-                                        int recent_start, const DecodeArgs& args, int b, StepRegs& s) {
-    const int row0 = 16 * sub;
+// Per-thread byte offsets inside a staged page, fixed for the whole kernel: every step's
+// code and RoPE rows start at a multiple of 8, so the 128-byte swizzle of a thread's
+// position does not depend on the step (step sub adds 2048, the second n-tile 1024).
+struct StageOffsets {
+    uint32_t code[4];      // codes of token r, channels 32q + 8i.. of group g
+    uint32_t kr0, kr1;     // RoPE channels 16q + 2i.. and 16q + 8 + 2i.. of token r
+};
+__device__ __forceinline__ StageOffsets stage_offsets(int q, int r, int i) {
+    StageOffsets o;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        const uint2 w = *reinterpret_cast<const uint2*>(pg + swz128(row0 + 8 * nt + r, 32 * g + 8 * i));
-        uint32_t t[4][2];
-        dequant_word(w.x, lut_lo, lut_hi, t);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) { s.bq[nt][kk][0] = t[kk][0]; s.bq[nt][kk][1] = t[kk][1]; }
-        dequant_word(w.y, lut_lo, lut_hi, t);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) { s.bq[nt][4 + kk][0] = t[kk][0]; s.bq[nt][4 + kk][1] = t[kk][1]; }
+    for (int g = 0; g < 4; ++g)
+        o.code[g] = r * 128 + (((2 * g + (q >> 1)) ^ r) << 4) + ((8 * q + 2 * i) & 15);
+    o.kr0 = (kKrRow + r) * 128 + (((2 * q) ^ r) << 4) + 4 * i;
+    o.kr1 = (kKrRow + r) * 128 + (((2 * q + 1) ^ r) << 4) + 4 * i;
+    return o;
+}
+
+// QK of one 16-token step for warp q, one channel group at a time.  Thread (r, i) builds
+// the x fragments of tokens r and r + 8 for channels 32q + 8i .. 32q + 8i + 7 of group g:
+// x[ks][nt][h] holds B-fragment k indices 2i + 8h + {0,1} of k-slice ks, which are
+// channels 32q + 8i + 2ks + h + {0, 4} (the query fragments use the same order).  Right
+// after its MMAs each group's fragments are transposed and stored as the PV A operand
+// (lanes 32q + 16ks + y for B-fragment k index y; ring columns 8g + c, where column 2i
+// holds tokens (2i, 2i+1) and column 2i + 1 tokens (8 + 2i, 9 + 2i)); the ring slot is
+// waited for before the first store.  Scores of the 16 heads x 16 tokens over this warp's
+// channels (plus its RoPE channels) go to sT with the token index XOR 8 * ((head >> 1) & 1)
+// (conflict-free stores and loads).  `pg` points at the step's first row.  PROT: some
+// token of the step is protected and takes its x from the bf16 side store (as fp16).
+template <bool PROT>
+__device__ __forceinline__ void qk_step(const uint8_t* pg, const StageOffsets& so, const uint2* lut,
+                                        float (*sT)[16], int q, int r, int i, const uint32_t (&qa)[4][2][4],
+                                        const uint32_t (&qra)[4], uint32_t a_taddr, uint32_t slot_bar,
+                                        unsigned slot_parity, bool slot_wait, volatile int* abort, int pos0,
+                                        int L, int recent_start, const DecodeArgs& args, int b) {
+    bool pa = false, pb = false;
+    const uint4* srca = nullptr;
+    const uint4* srcb = nullptr;
+    if (PROT) {
+        const int nslot = args.n_sink + args.n_recent;
+        const int p0 = pos0 + r, p1 = pos0 + 8 + r;
+        pa = p0 < L && (p0 < args.n_sink || p0 >= recent_start);
+        pb = p1 < L && (p1 < args.n_sink || p1 >= recent_start);
+        const int s0 = p0 < args.n_sink ? p0 : args.n_sink + p0 % max(args.n_recent, 1);
+        const int s1 = p1 < args.n_sink ? p1 : args.n_sink + p1 % max(args.n_recent, 1);
+        srca = reinterpret_cast<const uint4*>(args.prot + ((size_t)b * nslot + s0) * ROLAQ_D_C + 32 * q + 8 * i);
+        srcb = reinterpret_cast<const uint4*>(args.prot + ((size_t)b * nslot + s1) * ROLAQ_D_C + 32 * q + 8 * i);
     }
-    if (!FULL) {
-        // Protected tokens read their bf16 rotated content instead of the codes.
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int pos = pos0 + 8 * nt + r;
-            if (pos < L && (pos < args.n_sink || pos >= recent_start)) {
-                const int slot = pos < args.n_sink ? pos : args.n_sink + pos % args.n_recent;
-                const uint4* src = reinterpret_cast<const uint4*>(
-                    args.prot + ((size_t)b * (args.n_sink + args.n_recent) + slot) * ROLAQ_D_C + 128 * g + 32 * i);
-                uint32_t wv[16];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint4 v = src[q4];
-                    wv[4 * q4 + 0] = v.x; wv[4 * q4 + 1] = v.y; wv[4 * q4 + 2] = v.z; wv[4 * q4 + 3] = v.w;
-                }
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const int base = 16 * (ks >> 2), kk = ks & 3;
-                    const uint32_t sel = (kk & 1) ? 0x7632u : 0x5410u;
-                    s.bq[nt][ks][0] = prmt(wv[(base + kk) >> 1], wv[(base + 4 + kk) >> 1], sel);
-                    s.bq[nt][ks][1] = prmt(wv[(base + 8 + kk) >> 1], wv[(base + 12 + kk) >> 1], sel);
-                }
-            }
-        }
-    }
-    // metadata of the two tokens in each n-tile's column pair: mean, scale (kappa folded in)
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int t = row0 + 8 * nt + 2 * i + e;        // token row in the half page
-            const float2 ms = *reinterpret_cast<const float2*>(pg + swz128(32 + (t >> 2), (t & 3) * 32 + 8 * g));
-            if (FULL) {
-                s.mu[nt][e] = ms.x;
-                s.sc[nt][e] = ms.y * kappa;
-            } else {
-                const int tl = 8 * nt + 2 * i + e;
-                const int pos = pos0 + tl;
-                const bool valid = tl < nvalid;
-                const bool prot = pos < args.n_sink || pos >= recent_start;
-                s.mu[nt][e] = (valid && !prot) ? ms.x : 0.f;
-                s.sc[nt][e] = valid ? (prot ? 1.f : ms.y * kappa) : 0.f;
-            }
-        }
     float acc[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks)
+    for (int g = 0; g < 4; ++g) {
+        const uint32_t c0 = *reinterpret_cast<const uint16_t*>(pg + so.code[g]);
+        const uint32_t c1 = *reinterpret_cast<const uint16_t*>(pg + so.code[g] + 1024);
+        uint32_t t[4][2];
+        dequant_word2(c0 | (c1 << 16), lut[r * kLutStride + g], lut[(r + 8) * kLutStride + g], t);
+        uint32_t x[2][2][2];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) mma_bf16_16816(acc[nt], qa[ks], s.bq[nt][ks][0], s.bq[nt][ks][1]);
+        for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) x[ks][nt][h] = t[2 * ks + h][nt];
+        if (PROT) {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                if (nt == 0 ? pa : pb) {
+                    const uint4 u = (nt == 0 ? srca : srcb)[16 * g];
+                    x[0][nt][0] = pack_f16(bf16_lo(u.x), bf16_lo(u.z));
+                    x[0][nt][1] = pack_f16(bf16_hi(u.x), bf16_hi(u.z));
+                    x[1][nt][0] = pack_f16(bf16_lo(u.y), bf16_lo(u.w));
+                    x[1][nt][1] = pack_f16(bf16_hi(u.y), bf16_hi(u.w));
+                }
+            }
+        }
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) mma_f16_16816(acc[nt], qa[g][ks], x[ks][nt][0], x[ks][nt][1]);
+        if (g == 0) {
+            if (slot_wait) mbar_wait(slot_bar, slot_parity, abort);
+            tc_fence_after();
+        }
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+            const uint32_t v0 = movmatrix_trans(x[ks][0][0]);
+            const uint32_t v1 = movmatrix_trans(x[ks][1][0]);
+            const uint32_t v2 = movmatrix_trans(x[ks][0][1]);
+            const uint32_t v3 = movmatrix_trans(x[ks][1][1]);
+            asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1, %2, %3, %4};"
+                         :: "r"(a_taddr + ((uint32_t)(16 * ks) << 16) + 8 * g), "r"(v0), "r"(v1), "r"(v2),
+                            "r"(v3)
+                         : "memory");
+        }
+    }
+    const int sw = 8 * ((r >> 1) & 1);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-        // fold the group metadata: q.x = mean * sum(q_g) + scale * (q_g . level)
-        acc[nt][0] = fmaf(s.sc[nt][0], acc[nt][0], s.mu[nt][0] * qs0);
-        acc[nt][1] = fmaf(s.sc[nt][1], acc[nt][1], s.mu[nt][1] * qs0);
-        acc[nt][2] = fmaf(s.sc[nt][0], acc[nt][2], s.mu[nt][0] * qs1);
-        acc[nt][3] = fmaf(s.sc[nt][1], acc[nt][3], s.mu[nt][1] * qs1);
-        // RoPE part of the score for channels 16g..16g+15
-        const int row = 40 + row0 + 8 * nt + r;
-        const uint32_t kb0 = *reinterpret_cast<const uint32_t*>(pg + swz128(row, 32 * g + 4 * i));
-        const uint32_t kb1 = *reinterpret_cast<const uint32_t*>(pg + swz128(row, 32 * g + 16 + 4 * i));
+        // RoPE part of the score for channels 16q..16q+15
+        const uint32_t kb0 = *reinterpret_cast<const uint32_t*>(pg + so.kr0 + 1024 * nt);
+        const uint32_t kb1 = *reinterpret_cast<const uint32_t*>(pg + so.kr1 + 1024 * nt);
         mma_bf16_16816(acc[nt], qra, kb0, kb1);
-        const int tl = 8 * nt + 2 * i;
-        if (!FULL) {
-            if (tl >= nvalid) { acc[nt][0] = -INFINITY; acc[nt][2] = -INFINITY; }
-            if (tl + 1 >= nvalid) { acc[nt][1] = -INFINITY; acc[nt][3] = -INFINITY; }
-        }
-        *reinterpret_cast<float2*>(&sT[r][tl]) = make_float2(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<float2*>(&sT[r + 8][tl]) = make_float2(acc[nt][2], acc[nt][3]);
+        const int t = (8 * nt + 2 * i) ^ sw;
+        *reinterpret_cast<float2*>(&sT[r][t]) = make_float2(acc[nt][0], acc[nt][1]);
+        *reinterpret_cast<float2*>(&sT[r + 8][t]) = make_float2(acc[nt][2], acc[nt][3]);
     }
 }
 
-// Softmax for heads 4g..4g+3 over one step's 16 tokens: lane (head hh, token pair jj).
-// The reference max m_ref moves only when a score exceeds it by more than kRescaleLog2
-// (one warp vote in the common case; shuffles only when some head moves), so the
-// probabilities relative to m_ref stay below 2^kRescaleLog2.  l_part is this lane's share
-// of the row sum, reduced over the 8 lanes of the head at the end.
-__device__ __forceinline__ void softmax_step(float (*sT)[16][kSStride], float (*sP)[kSStride], float* sAl,
-                                             int hh, int jj, float scale_log2, float& m_ref, float& l_part) {
-    float2 v0 = *reinterpret_cast<const float2*>(&sT[0][hh][2 * jj]);
-    float2 v1 = *reinterpret_cast<const float2*>(&sT[1][hh][2 * jj]);
-    float2 v2 = *reinterpret_cast<const float2*>(&sT[2][hh][2 * jj]);
-    float2 v3 = *reinterpret_cast<const float2*>(&sT[3][hh][2 * jj]);
-    const float s0 = ((v0.x + v1.x) + (v2.x + v3.x)) * scale_log2;
-    const float s1 = ((v0.y + v1.y) + (v2.y + v3.y)) * scale_log2;
+// Softmax of one step for head hh (of the 16-head chunk), tokens 2jj, 2jj+1.  The
+// reference max m_ref moves only when a score exceeds it by more than kRescaleLog2
+// (one warp vote in the common case), so probabilities relative to m_ref stay below
+// 2^kRescaleLog2.  The fp16 probabilities go to the B tile at K positions
+// 4jj, 4jj+1 (jj < 4) or 4(jj-4)+2, +3, matching the A tile's column order.
+__device__ __forceinline__ void softmax_step(const float (*sT)[16][16], uint8_t* Pt, float* sAl, int* resc,
+                                             int hh, int jj, int nvalid, float scale_log2, bool first,
+                                             float& m_ref, float& l_part) {
+    const int t = (2 * jj) ^ (8 * ((hh >> 1) & 1));
+    const float2 v0 = *reinterpret_cast<const float2*>(&sT[0][hh][t]);
+    const float2 v1 = *reinterpret_cast<const float2*>(&sT[1][hh][t]);
+    const float2 v2 = *reinterpret_cast<const float2*>(&sT[2][hh][t]);
+    const float2 v3 = *reinterpret_cast<const float2*>(&sT[3][hh][t]);
+    float s0 = ((v0.x + v1.x) + (v2.x + v3.x)) * scale_log2;
+    float s1 = ((v0.y + v1.y) + (v2.y + v3.y)) * scale_log2;
+    if (2 * jj >= nvalid) s0 = -INFINITY;
+    if (2 * jj + 1 >= nvalid) s1 = -INFINITY;
     float alpha = 1.f;
     const bool up = fmaxf(s0, s1) > m_ref + kRescaleLog2 || (m_ref == -INFINITY && fmaxf(s0, s1) > -INFINITY);
     if (__any_sync(0xffffffffu, up)) {
@@ -317,63 +366,56 @@ __device__ __forceinline__ void softmax_step(float (*sT)[16][kSStride], float (*
     const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
     const float p0 = ex2(s0 - mu), p1 = ex2(s1 - mu);
     l_part += p0 + p1;
-    *reinterpret_cast<float2*>(&sP[hh][2 * jj]) = make_float2(p0, p1);
+    const int kp = jj < 4 ? 4 * jj : 4 * (jj - 4) + 2;
+    const int off = (hh >> 3) * 256 + (kp >> 3) * 128 + (hh & 7) * 16 + (kp & 7) * 2;
+    *reinterpret_cast<uint32_t*>(Pt + off) = pack_f16(p0, p1);
     if (jj == 0) sAl[hh] = alpha;
+    if (alpha != 1.f && !first) *resc = 1;
 }
 
-// PV inputs of one step (probabilities of the fragment rows/columns, rescale factors),
-// read before the softmax of the next step writes its own buffers.
-struct PvIn {
-    float2 p00, p10, p02, p12;
-    float al0, al1;
-};
-__device__ __forceinline__ PvIn pv_load(const float (*__restrict__ sP)[kSStride], const float* __restrict__ sAl,
-                                        int r, int i) {
-    PvIn v;
-    const int tl = 2 * i;
-    v.p00 = *reinterpret_cast<const float2*>(&sP[r][tl]);
-    v.p10 = *reinterpret_cast<const float2*>(&sP[r + 8][tl]);
-    v.p02 = *reinterpret_cast<const float2*>(&sP[r][tl + 8]);
-    v.p12 = *reinterpret_cast<const float2*>(&sP[r + 8][tl + 8]);
-    v.al0 = sAl[r];
-    v.al1 = sAl[r + 8];
-    return v;
-}
-
-// PV for one step: O_g[h, ch] += sum_t p * scale_t * level + (sum_t p * mean_t).
-__device__ __forceinline__ void pv_step(const PvIn& v, const StepRegs& s, float (&o)[8][2][4], float& u0,
-                                        float& u1) {
-    if (__any_sync(0xffffffffu, v.al0 != 1.f || v.al1 != 1.f)) {
+// PV of team step jp, called by all 128 threads of the team after the step barrier that
+// follows softmax(jp).  When some head's running max moved at jp, every warp first scales
+// its lanes of O (the PV of step jp-1 has completed: its ring slot was waited for), then
+// lane 0 of the team's first warp issues the four group MMAs and commits them to the
+// slot's barrier.
+__device__ __forceinline__ void pv_issue(DecodeSmem& sm, int team, int q, int lane, int jp, uint32_t tmem,
+                                         int bar_id) {
+    const int buf = jp & 1;
+    if (sm.resc[team][buf]) {
+        tc_fence_after();
+        const uint32_t ocol = tmem + ((uint32_t)(32 * q) << 16) + team * kTeamCols;
+#pragma unroll 1
+        for (int g = 0; g < 4; ++g) {
+            uint32_t u[16];
+            tmem_ld16(ocol + 16 * g, u);
+            tmem_ld_wait();
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                o[ks][hf][0] *= v.al0; o[ks][hf][1] *= v.al0;
-                o[ks][hf][2] *= v.al1; o[ks][hf][3] *= v.al1;
-            }
-        u0 *= v.al0;
-        u1 *= v.al1;
+            for (int h = 0; h < 16; ++h) u[h] = __float_as_uint(__uint_as_float(u[h]) * sm.sAl[team][buf][h]);
+            tmem_st16(ocol + 16 * g, u);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        named_bar_sync(bar_id, 128);
+        if (q == 0 && lane == 0) sm.resc[team][buf] = 0;
     }
-    u0 += v.p00.x * s.mu[0][0] + v.p00.y * s.mu[0][1] + v.p02.x * s.mu[1][0] + v.p02.y * s.mu[1][1];
-    u1 += v.p10.x * s.mu[0][0] + v.p10.y * s.mu[0][1] + v.p12.x * s.mu[1][0] + v.p12.y * s.mu[1][1];
-    uint32_t pa[4];
-    pa[0] = pack_bf16(v.p00.x * s.sc[0][0], v.p00.y * s.sc[0][1]);
-    pa[1] = pack_bf16(v.p10.x * s.sc[0][0], v.p10.y * s.sc[0][1]);
-    pa[2] = pack_bf16(v.p02.x * s.sc[1][0], v.p02.y * s.sc[1][1]);
-    pa[3] = pack_bf16(v.p12.x * s.sc[1][0], v.p12.y * s.sc[1][1]);
+    if (q == 0 && lane == 0) {
+        tc_fence_after();
+        const int slot = jp % kRing;
+        const uint32_t obase = tmem + team * kTeamCols;
+        const uint32_t abase = obase + kRingCol + 32 * slot;
+        const uint64_t bd = umma_desc_plain(smem_u32(sm.P[team][slot]));
 #pragma unroll
-    for (int ks = 0; ks < 8; ++ks)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-            mma_bf16_16816(o[ks][hf], pa, movmatrix_trans(s.bq[0][ks][hf]), movmatrix_trans(s.bq[1][ks][hf]));
+        for (int g = 0; g < 4; ++g) umma_ts(obase + 16 * g, abase + 8 * g, bd, jp > 0 ? 1u : 0u);
+        umma_commit(smem_u32(&sm.pvbar[team][slot]));
+    }
 }
 
 __global__ void __launch_bounds__(kDecodeThreads, 1)
-rolaq_decode_split(const __grid_constant__ CUtensorMap map32, const __grid_constant__ CUtensorMap map8,
-                   const DecodeArgs args) {
+rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArgs args) {
     extern __shared__ uint8_t smem_raw[];
-    DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // offset the __shared__ array itself (not an integer address) so that every access
+    // stays a shared-memory access
+    DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int hc = blockIdx.y;                 // 16-head chunk
 
@@ -386,142 +428,201 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map32, const __grid_const
         }
     }
     if (threadIdx.x == 32) {
-        for (int t = 0; t < 2; ++t)
-            for (int s = 0; s < kNStage; ++s) mbar_init(smem_u32(&sm.full[t][s]), 1);
+        for (int t = 0; t < kTeams; ++t) {
+            for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&sm.full[t][s]), 1);
+            for (int s = 0; s < kRing; ++s) mbar_init(smem_u32(&sm.pvbar[t][s]), 1);
+            sm.resc[t][0] = sm.resc[t][1] = 0;
+        }
         sm.abort = 0;
         fence_mbar_init();
-        prefetch_tmap(&map32);
-        prefetch_tmap(&map8);
+        prefetch_tmap(&map_page);
     }
     __syncthreads();
     const int b = sm.plan[0];
     if (b < 0) return;                         // item past the end of the plan
     const int first_page = sm.plan[1], n_pages = sm.plan[2];
     const int L = args.seq_lens[b];
-    const int item = blockIdx.x;
-    const int team = warp >> 2, g = warp & 3;
-    const bool producer = (g == 0) && (lane == 0);
-    if (producer)
-        for (int k = 0; k < n_pages && k < kNStage; ++k)
-            load_half_page(sm, &map32, &map8, args, team, b, first_page + k, k);
+    const int team = warp >> 2, q = warp & 3;
+    const int tid = threadIdx.x & 127;
+    const bool leader = (q == 0) && (lane == 0);
+    const int n_team = n_pages > team ? (n_pages - team + kTeams - 1) / kTeams : 0;
+    const int J = n_team * (kPageTok / kStepTok);
+    auto page_of = [&](int k) { return first_page + team + kTeams * k; };
+    if (leader)
+        for (int k = 0; k < n_team && k < kStages; ++k) load_page(sm, &map_page, args, team, b, page_of(k), k);
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
+                     :: "r"(smem_u32(&sm.tmem_base)) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
 
     const int r = lane >> 2, i = lane & 3;     // mma fragment row group / thread in group
     const int h0 = hc * 16;
-    const __nv_bfloat16* qrow0 = args.q + ((size_t)b * args.heads + h0 + r) * ROLAQ_D_C + 128 * g;
-    const __nv_bfloat16* qrow1 = qrow0 + 8 * ROLAQ_D_C;
-
-    // Query fragments for this warp's group, in the qk_channel order; row sums of q_g.
-    uint32_t qa[8][4];
-    float qs0 = 0.f, qs1 = 0.f;
+    // Query fragments (fp16) in the channel order of qk_step.
+    uint32_t qa[4][2][4];
+    {
+        const uint16_t* u0 = reinterpret_cast<const uint16_t*>(args.q + ((size_t)b * args.heads + h0 + r) * ROLAQ_D_C);
+        const uint16_t* u1 = u0 + 8 * ROLAQ_D_C;
+        float qmax = 0.f;
+        auto f = [&](const uint16_t* u, int c) {
+            const float v = __uint_as_float((uint32_t)u[c] << 16);
+            qmax = fmaxf(qmax, fabsf(v));
+            return v;
+        };
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-        const int c0 = qk_channel(s, 2 * i), c1 = qk_channel(s, 2 * i + 1);
-        const int c2 = qk_channel(s, 2 * i + 8), c3 = qk_channel(s, 2 * i + 9);
-        const float v00 = __bfloat162float(qrow0[c0]), v01 = __bfloat162float(qrow0[c1]);
-        const float v02 = __bfloat162float(qrow0[c2]), v03 = __bfloat162float(qrow0[c3]);
-        const float v10 = __bfloat162float(qrow1[c0]), v11 = __bfloat162float(qrow1[c1]);
-        const float v12 = __bfloat162float(qrow1[c2]), v13 = __bfloat162float(qrow1[c3]);
-        qa[s][0] = pack_bf16(v00, v01);
-        qa[s][1] = pack_bf16(v10, v11);
-        qa[s][2] = pack_bf16(v02, v03);
-        qa[s][3] = pack_bf16(v12, v13);
-        qs0 += (v00 + v01) + (v02 + v03);
-        qs1 += (v10 + v11) + (v12 + v13);
+        for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+                const int c = 128 * g + 32 * q + 8 * i + 2 * ks;
+                qa[g][ks][0] = pack_f16(f(u0, c), f(u0, c + 4));
+                qa[g][ks][1] = pack_f16(f(u1, c), f(u1, c + 4));
+                qa[g][ks][2] = pack_f16(f(u0, c + 1), f(u0, c + 5));
+                qa[g][ks][3] = pack_f16(f(u1, c + 1), f(u1, c + 5));
+            }
+        if (!(qmax < kF16Max)) raise_status(ROLAQ_STATUS_RANGE);
     }
-    qs0 += __shfl_xor_sync(0xffffffffu, qs0, 1);
-    qs0 += __shfl_xor_sync(0xffffffffu, qs0, 2);
-    qs1 += __shfl_xor_sync(0xffffffffu, qs1, 1);
-    qs1 += __shfl_xor_sync(0xffffffffu, qs1, 2);
     uint32_t qra[4];
     {
         const uint32_t* r0 = reinterpret_cast<const uint32_t*>(
-            args.qr + ((size_t)b * args.heads + h0 + r) * ROLAQ_D_R + 16 * g);
+            args.qr + ((size_t)b * args.heads + h0 + r) * ROLAQ_D_R + 16 * q);
         const uint32_t* r1 = r0 + 8 * ROLAQ_D_R / 2;
         qra[0] = r0[i];
         qra[1] = r1[i];
         qra[2] = r0[4 + i];
         qra[3] = r1[4 + i];
     }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
 
-    float o[8][2][4];
-#pragma unroll
-    for (int s = 0; s < 8; ++s)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) o[s][hf][c] = 0.f;
-    float u0 = 0.f, u1 = 0.f;                 // mean-term accumulators, rows r and r+8
-    float m_ref = -INFINITY, l_part = 0.f;    // softmax state of head 4g + lane/8 (this lane's share)
-    const int hh = 4 * g + (lane >> 3), jj = lane & 7;
-
-    const uint32_t lut_lo = args.lut_lo, lut_hi = args.lut_hi;
+    const int hh = 4 * q + (lane >> 3), jj = lane & 7;   // softmax: head, token pair
+    const int bar_id = 1 + team;
     const bool protect = args.n_sink > 0 || args.n_recent > 0;
     const int recent_start = L - args.n_recent;
-    const int bar_id = 1 + team;
+    const float lva = args.level_a, lvb = args.level_b;
+    const uint32_t a_lane = tmem + ((uint32_t)(32 * q) << 16) + team * kTeamCols + kRingCol;
+    const StageOffsets so = stage_offsets(q, r, i);
+    float m_ref = -INFINITY, l_part = 0.f;
 
-    // QK of step (page k, sub) into regs: waits for the stage when sub == 0.
-    auto qk = [&](int k, int sub, int buf, StepRegs& regs) {
-        const int st = k % kNStage;
-        if (sub == 0) mbar_wait(smem_u32(&sm.full[team][st]), (k / kNStage) & 1, &sm.abort);
-        const int pos0 = (first_page + k) * kPageTok + 32 * team + kStepTok * sub;
+    if (J > 0 && tid < 64) {
+        mbar_wait(smem_u32(&sm.full[team][0]), 0, &sm.abort);
+        lut_prep(sm.stage[team][0], sm.valid[team][0] != 0, 0, tid >> 2, tid & 3,
+                 page_of(0) * kPageTok + (tid >> 2), L, lva, lvb, &sm.lut[team][0][0][0]);
+    }
+    named_bar_sync(bar_id, 128);
+
+    for (int j = 0; j < J; ++j) {
+        const int k = j >> 2, sub = j & 3, st = k % kStages;
+        if (sub == 0) mbar_wait(smem_u32(&sm.full[team][st]), (k / kStages) & 1, &sm.abort);
+        const uint8_t* pg = sm.stage[team][st];
+        const int pos0 = page_of(k) * kPageTok + kStepTok * sub;
         const int nvalid = sm.valid[team][st] ? min(max(L - pos0, 0), kStepTok) : 0;
-        const bool mixed = protect && (pos0 < args.n_sink || pos0 + kStepTok > recent_start);
-        if (nvalid == kStepTok && !mixed)
-            qk_step<true>(sm.stage[team][st], sub, sm.sT[team][buf][g], r, i, g, lut_lo, lut_hi, args.kappa,
-                          qa, qra, qs0, qs1, kStepTok, pos0, L, recent_start, args, b, regs);
+        const bool prot = protect && (pos0 < args.n_sink || pos0 + kStepTok > recent_start);
+        const int slot = j % kRing;
+        const uint32_t slot_bar = smem_u32(&sm.pvbar[team][slot]);
+        const unsigned slot_par = (unsigned)(((j - kRing) / kRing) & 1);
+        const uint8_t* pgs = pg + sub * (kStepTok * 128);
+        // QK of step j; its A tile goes to ring slot j % kRing once PV(j - kRing) has read it
+        if (prot)
+            qk_step<true>(pgs, so, &sm.lut[team][j & 1][0][0], sm.sT[team][j & 1][q], q, r, i, qa, qra,
+                          a_lane + 32 * slot, slot_bar, slot_par, j >= kRing, &sm.abort, pos0, L, recent_start,
+                          args, b);
         else
-            qk_step<false>(sm.stage[team][st], sub, sm.sT[team][buf][g], r, i, g, lut_lo, lut_hi, args.kappa,
-                           qa, qra, qs0, qs1, nvalid, pos0, L, recent_start, args, b, regs);
-    };
-
-    StepRegs ra, rb;
-    if (n_pages > 0) {
-        qk(0, 0, 0, ra);
+            qk_step<false>(pgs, so, &sm.lut[team][j & 1][0][0], sm.sT[team][j & 1][q], q, r, i, qa, qra,
+                           a_lane + 32 * slot, slot_bar, slot_par, j >= kRing, &sm.abort, pos0, L, recent_start,
+                           args, b);
+        tmem_st_wait();
+        tc_fence_before();
+        // lookup pairs of step j + 1
+        if (j + 1 < J && tid < 64) {
+            const int jn = j + 1, kn = jn >> 2, subn = jn & 3, stn = kn % kStages;
+            if (subn == 0) mbar_wait(smem_u32(&sm.full[team][stn]), (kn / kStages) & 1, &sm.abort);
+            lut_prep(sm.stage[team][stn], sm.valid[team][stn] != 0, subn, tid >> 2, tid & 3,
+                     page_of(kn) * kPageTok + kStepTok * subn + (tid >> 2), L, lva, lvb,
+                     &sm.lut[team][jn & 1][0][0]);
+        }
         named_bar_sync(bar_id, 128);
-        softmax_step(sm.sT[team][0], sm.sP[team][0], sm.sAl[team][0], hh, jj, args.scale_log2, m_ref, l_part);
+        // page k is fully read after its last step: refill its stage
+        if (leader && sub == 3 && k + kStages < n_team)
+            load_page(sm, &map_page, args, team, b, page_of(k + kStages), k + kStages);
+        if (j >= 1) pv_issue(sm, team, q, lane, j - 1, tmem, bar_id);
+        softmax_step(sm.sT[team][j & 1], sm.P[team][slot], sm.sAl[team][j & 1], &sm.resc[team][j & 1], hh, jj,
+                     nvalid, args.scale_log2, j == 0, m_ref, l_part);
+        fence_proxy_async_smem();
     }
-    for (int k = 0; k < n_pages; ++k) {
-        // step 2k+1 (second 16 tokens of page k) into rb; PV of step 2k from ra
-        qk(k, 1, 1, rb);
+    if (J > 0) {
+        if (J >= kRing) mbar_wait(smem_u32(&sm.pvbar[team][J % kRing]), ((J - kRing) / kRing) & 1, &sm.abort);
         named_bar_sync(bar_id, 128);
-        // every warp of the team is done reading stage k: refill it
-        if (producer && k + kNStage < n_pages)
-            load_half_page(sm, &map32, &map8, args, team, b, first_page + k + kNStage, k + kNStage);
-        const PvIn va = pv_load(sm.sP[team][0], sm.sAl[team][0], r, i);
-        softmax_step(sm.sT[team][1], sm.sP[team][1], sm.sAl[team][1], hh, jj, args.scale_log2, m_ref, l_part);
-        pv_step(va, ra, o, u0, u1);
-        // step 2k+2 (first 16 tokens of page k+1) into ra; PV of step 2k+1 from rb
-        const bool more = k + 1 < n_pages;
-        if (more) qk(k + 1, 0, 0, ra);
-        named_bar_sync(bar_id, 128);
-        const PvIn vb = pv_load(sm.sP[team][1], sm.sAl[team][1], r, i);
-        if (more)
-            softmax_step(sm.sT[team][0], sm.sP[team][0], sm.sAl[team][0], hh, jj, args.scale_log2, m_ref, l_part);
-        pv_step(vb, rb, o, u0, u1);
+        pv_issue(sm, team, q, lane, J - 1, tmem, bar_id);
+        mbar_wait(smem_u32(&sm.pvbar[team][(J - 1) % kRing]), ((J - 1) / kRing) & 1, &sm.abort);
+        tc_fence_after();
     }
-
-    // ---- write this team's partial: O + mean term, and (m, l) per head ---------
-    u0 += __shfl_xor_sync(0xffffffffu, u0, 1);
-    u0 += __shfl_xor_sync(0xffffffffu, u0, 2);
-    u1 += __shfl_xor_sync(0xffffffffu, u1, 1);
-    u1 += __shfl_xor_sync(0xffffffffu, u1, 2);
     l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
     l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
     l_part += __shfl_xor_sync(0xffffffffu, l_part, 4);
-    const size_t part = (size_t)item * 2 + team;
-    float* out0 = args.ws_o + (part * args.heads + h0 + r) * ROLAQ_D_C + 128 * g;
-    float* out1 = out0 + 8 * ROLAQ_D_C;
+    if (jj == 0) sm.team_ml[team][hh] = make_float2(m_ref, l_part);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- merge the teams: warp q of team t writes channel groups t, t + kTeams, ... ----
+    {
+        float Mx[16];
 #pragma unroll
-    for (int s = 0; s < 8; ++s)
+        for (int h = 0; h < 16; ++h) {
+            float m = sm.team_ml[0][h].x;
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
+            for (int t = 1; t < kTeams; ++t) m = fmaxf(m, sm.team_ml[t][h].x);
+            Mx[h] = m;
+        }
+        const int ks = lane >> 4, y = lane & 15;
+        const int chq = 32 * q + 8 * ((y & 7) >> 1) + 4 * (y & 1) + 2 * ks + (y >> 3);
+#pragma unroll 1
+        for (int g = team; g < 4; g += kTeams) {
+            float acc[16];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int ch = 32 * i + 16 * (s >> 2) + 8 * hf + 4 * e + (s & 3);
-                out0[ch] = o[s][hf][e] + u0;
-                out1[ch] = o[s][hf][2 + e] + u1;
+            for (int h = 0; h < 16; ++h) acc[h] = 0.f;
+#pragma unroll 1
+            for (int t = 0; t < kTeams; ++t) {
+                float w[16];
+                bool any = false;
+#pragma unroll
+                for (int h = 0; h < 16; ++h) {
+                    const float m = sm.team_ml[t][h].x;
+                    w[h] = (m == -INFINITY) ? 0.f : ex2(m - Mx[h]);
+                    any |= w[h] != 0.f;
+                }
+                if (any) {                           // the same for every lane of the warp
+                    uint32_t u[16];
+                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + t * kTeamCols + 16 * g, u);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < 16; ++h)
+                        if (w[h] != 0.f) acc[h] = fmaf(w[h], __uint_as_float(u[h]), acc[h]);
+                }
             }
-    if (jj == 0) args.ws_ml[part * args.heads + h0 + hh] = make_float2(m_ref, l_part);
+            float* dst = args.ws_o + ((size_t)blockIdx.x * args.heads + h0) * ROLAQ_D_C + 128 * g + chq;
+#pragma unroll
+            for (int h = 0; h < 16; ++h) dst[(size_t)h * ROLAQ_D_C] = acc[h];
+        }
+        if (team == 0 && q == 0 && lane < 16) {
+            float m = sm.team_ml[0][lane].x;
+            for (int t = 1; t < kTeams; ++t) m = fmaxf(m, sm.team_ml[t][lane].x);
+            float l = 0.f;
+            for (int t = 0; t < kTeams; ++t) {
+                const float2 ml = sm.team_ml[t][lane];
+                if (ml.x != -INFINITY) l += ex2(ml.x - m) * ml.y;
+            }
+            args.ws_ml[(size_t)blockIdx.x * args.heads + h0 + lane] = make_float2(m, l);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" :: "r"(tmem) : "memory");
+    }
 }
 
 // ---- merge --------------------------------------------------------------------
@@ -547,7 +648,7 @@ rolaq_decode_merge(const float* __restrict__ ws_o, const float2* __restrict__ ws
         if (lane == 0) { s_plan[0] = pi.item_offset; s_plan[1] = pi.n_items; }
     }
     __syncthreads();
-    const int p0 = 2 * s_plan[0], np = 2 * s_plan[1];
+    const int p0 = s_plan[0], np = s_plan[1];
     // max over partials
     float M = -INFINITY;
     for (int p = threadIdx.x; p < np; p += kMergeThreads) M = fmaxf(M, ws_ml[(size_t)(p0 + p) * heads + h].x);

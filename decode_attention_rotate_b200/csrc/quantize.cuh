@@ -75,16 +75,6 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t da, uint64_t
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         :: "r"(tmem_d), "l"(da), "l"(db), "r"(kQIdesc), "r"(acc) : "memory");
 }
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-                 :: "r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
 // 32 lanes x 32 columns of fp32 from TMEM, one row (lane) per thread.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     uint32_t* u = reinterpret_cast<uint32_t*>(v);
@@ -98,9 +88,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
           "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]), "=r"(u[25]),
           "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
         : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld_wait() {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 // 32 columns of y = chain A + chain B (fp32 add of the two K-half accumulators).
 __device__ __forceinline__ void load_y32(uint32_t col_a, uint32_t col_b, float (&y)[32]) {
@@ -177,8 +164,9 @@ __global__ void __launch_bounds__(kQThreads, 1)
 rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
                       const __grid_constant__ CUtensorMap map_r, const QuantArgs args) {
     extern __shared__ uint8_t smem_raw[];
-    QuantSmem& sm = *reinterpret_cast<QuantSmem*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // offset the __shared__ array itself (not an integer address) so that every access
+    // stays a shared-memory access
+    QuantSmem& sm = *reinterpret_cast<QuantSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = (args.n + kQTileM - 1) / kQTileM;
 

@@ -67,39 +67,6 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, void* base, uint64_t in
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// bf16 bit pattern of an fp32 value, round to nearest even (finite inputs).
-uint16_t bf16_bits(float x) {
-    uint32_t u;
-    memcpy(&u, &x, 4);
-    u += 0x7FFFu + ((u >> 16) & 1u);
-    return (uint16_t)(u >> 16);
-}
-
-// bf16 level pair for the decode MMAs.  Plain bf16(a), bf16(b) are off by up to 2^-9,
-// which moves every score by that much.  Instead pick B = 1 + m/128 and A = bf16(B a/b)
-// over the 128 mantissas m so that A / B matches a / b (typically to ~1e-5; near
-// a/b = 1/4 the choices alias and it degrades to ~1e-3), and return kappa, the
-// geometric mean of a/A and b/B, which splits the remaining ratio error evenly between
-// the two levels.  kappa is folded into the per-token scale.
-void level_encoding(float a, float b, uint16_t* a_bits, uint16_t* b_bits, float* kappa) {
-    const double rho = (double)a / (double)b;
-    double best = 1e30;
-    for (int m = 0; m < 128; ++m) {
-        const double B = 1.0 + m / 128.0;
-        const uint16_t ab = bf16_bits((float)(rho * B));
-        uint32_t u = (uint32_t)ab << 16;
-        float A;
-        memcpy(&A, &u, 4);
-        const double err = fabs((double)A / B - rho);
-        if (err < best) {
-            best = err;
-            *a_bits = ab;
-            *b_bits = bf16_bits((float)B);
-            *kappa = (float)sqrt(((double)a / A) * ((double)b / B));
-        }
-    }
-}
-
 int check_cache(const rolaq_cache* c) {
     if (!c || !c->pages_dev || !c->page_table_dev || c->num_pages <= 0 || c->batch <= 0 ||
         c->max_pages_per_seq <= 0)
@@ -126,8 +93,8 @@ int decode_target_items(int heads) {
 
 size_t decode_ws_bytes(int batch, int heads) {
     const size_t items = (size_t)decode_target_items(heads) + (size_t)batch;
-    const size_t o = items * 2 * heads * ROLAQ_D_C * sizeof(float);
-    const size_t ml = items * 2 * heads * sizeof(float2);
+    const size_t o = items * heads * ROLAQ_D_C * sizeof(float);
+    const size_t ml = items * heads * sizeof(float2);
     return o + ml;
 }
 
@@ -270,13 +237,11 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
     if (!isfinite(sm_scale)) return ROLAQ_EINVAL;
     if (workspace_bytes < decode_ws_bytes(batch, heads)) return ROLAQ_ENOSPACE;
 
-    // The pool as rows of 128 B; boxes of 32 rows (codes, k_R) and 8 rows (metadata).
-    CUtensorMap map32, map8;
+    // The pool as rows of 128 B; one box is a whole page (144 rows).
+    CUtensorMap map_page;
     const uint64_t rows = (uint64_t)cache->num_pages * (ROLAQ_PAGE_BYTES / 128);
-    if (!encode_2d(&map32, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache->pages_dev, 128, rows, 128, 128, 32,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&map8, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache->pages_dev, 128, rows, 128, 128, 8,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_2d(&map_page, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache->pages_dev, 128, rows, 128, 128,
+                   ROLAQ_PAGE_BYTES / 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return ROLAQ_ECUDA;
 
     const int target = decode_target_items(heads);
@@ -294,22 +259,12 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
     a.batch = batch;
     a.heads = heads;
     a.scale_log2 = sm_scale * 1.4426950408889634f;
-    uint16_t abits = 0, bbits = 0;
-    float kappa = 1.f;
-    level_encoding(p->level_a, p->level_b, &abits, &bbits, &kappa);
-    const uint16_t lv[4] = {(uint16_t)(bbits | 0x8000u), (uint16_t)(abits | 0x8000u), abits, bbits};
-    uint32_t lo = 0, hi = 0;
-    for (int c = 0; c < 4; ++c) {
-        lo |= (uint32_t)(lv[c] & 0xFFu) << (8 * c);
-        hi |= (uint32_t)(lv[c] >> 8) << (8 * c);
-    }
-    a.lut_lo = lo;
-    a.lut_hi = hi;
-    a.kappa = kappa;
+    a.level_a = p->level_a;
+    a.level_b = p->level_b;
     a.target_items = target;
     a.ws_o = reinterpret_cast<float*>(workspace_dev);
     a.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace_dev) +
-                                        (size_t)items_cap * 2 * heads * ROLAQ_D_C * sizeof(float));
+                                        (size_t)items_cap * heads * ROLAQ_D_C * sizeof(float));
 
     const size_t smem = sizeof(DecodeSmem) + 1024;
     static std::once_flag attr_once;
@@ -317,7 +272,7 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
         cudaFuncSetAttribute(rolaq_decode_split, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     });
     cudaStream_t s = (cudaStream_t)stream;
-    rolaq_decode_split<<<dim3(items_cap, heads / 16), kDecodeThreads, smem, s>>>(map32, map8, a);
+    rolaq_decode_split<<<dim3(items_cap, heads / 16), kDecodeThreads, smem, s>>>(map_page, a);
     if ((rc = launch_status())) return rc;
     rolaq_decode_merge<<<dim3(batch, heads), kMergeThreads, 0, s>>>(a.ws_o, a.ws_ml, seq_lens_dev, batch, heads,
                                                          target, out_dev, lse_dev);

@@ -26,6 +26,7 @@ RSPLIT_BYTES = 3 * 512 * 512 * 2
 STATUS_BAD_PAGE = 1
 STATUS_BAD_SLOT = 2
 STATUS_TIMEOUT = 4
+STATUS_RANGE = 8
 
 
 class RolaqError(RuntimeError):

@@ -89,6 +89,8 @@ extern "C" {
 #define ROLAQ_STATUS_BAD_PAGE   1  /* page-table entry < 0 or >= num_pages (skipped)  */
 #define ROLAQ_STATUS_BAD_SLOT   2  /* append target outside its request's pages       */
 #define ROLAQ_STATUS_TIMEOUT    4  /* a pipeline wait gave up (results of that call invalid) */
+#define ROLAQ_STATUS_RANGE      8  /* a decoded x or a query element beyond the fp16 range
+                                      (|x|, |q| >= 65504): that decode result is invalid  */
 
 /* Cache descriptor.  Plain data; the caller owns every buffer it points to.
  *   pages_dev       page pool, num_pages * ROLAQ_PAGE_BYTES bytes, 1024-B aligned.
@@ -163,7 +165,11 @@ size_t rolaq_decode_workspace_bytes(int batch, int heads);
  * (may be NULL).  heads must be a positive multiple of 16, batch <= cache->batch.
  * L == 0 gives out = 0 and lse = -inf.  workspace_dev (16-B aligned) must hold
  * rolaq_decode_workspace_bytes(batch, heads) bytes; it is scratch owned by the caller
- * and needs no initialisation.  Split-K over the sequence with a log-sum-exp merge.   */
+ * and needs no initialisation.  Split-K over the sequence with a log-sum-exp merge.
+ * Arithmetic: x_t, q_c_rot and the probabilities enter the tensor-core products as fp16
+ * (k_R and q_R as bf16); scores, sums and out accumulate in fp32.  A token whose
+ * |mean| + scale * level_b, or a query element whose magnitude, reaches 65504 sets
+ * ROLAQ_STATUS_RANGE.                                                                */
 int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
                       const void* q_c_rot_dev, const void* q_R_dev,
                       const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
