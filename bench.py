@@ -33,11 +33,12 @@ METRIC = "2-bit MLA decode: cache GB/s & % HBM roofline; quantize-append tokens/
 SM_SCALE = 1.0 / math.sqrt(192.0)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-# DRAM bytes (read + write) per decode launch of the bench workload, from the ncu capture
-# summarised in profiles/decode_split_4x128k_h16.md (4 x 131,072 tokens): reads 151.18 MB
-# scale with the tokens (x2 here), the 5.79 MB of split-K partials depend only on the item
-# count, which is the same; None whenever the kernel has changed since that capture.
-DECODE_TRAFFIC_PER_LAUNCH = None
+# DRAM bytes (read + write) of the split kernel per decode launch of the bench workload,
+# from the ncu capture summarised in profiles/decode_split_4x128k_h16.md (4 x 131,072
+# tokens): the 151.51 MB of reads scale with the tokens (x2 here); the 4.97 MB of split-K
+# partials depend only on the item count, which is the same.  None whenever the kernel
+# has changed since that capture.
+DECODE_TRAFFIC_PER_LAUNCH = 2 * 151.51e6 + 4.97e6
 
 
 def peaks():
@@ -283,7 +284,7 @@ def run_ours(args, rank, world, dev):
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16+bf16",
         "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_lens[0], "heads": w.heads,
                    "layers": w.layers, "cache_bytes_per_step": step_bytes,
@@ -291,7 +292,8 @@ def run_ours(args, rank, world, dev):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "traffic": DECODE_TRAFFIC_PER_LAUNCH,
-                     "kernel": "decode (split + merge launches)", "peak_source": src,
+                     "kernel": "decode call (split + merge launches); traffic: split kernel",
+                     "peak_source": src,
                      "bytes_per_launch": dec_bytes, "ms_per_launch": round(dec_ms, 4),
                      "frac_of_8tbs": round(achieved / 8000.0, 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
