@@ -365,14 +365,19 @@ namespace rolaq {
 // ---- small appends --------------------------------------------------------------
 // A decode step appends one token per request: a few tokens per call.  The tensor-core
 // kernel above would stream all of R through a single CTA for them, so small calls use
-// this kernel instead: one CTA of 16 warps per (group, 8 tokens).  Warp w computes output
-// coordinates 128g + 8w .. +7: for each, the 32 lanes read the three R-plane rows
-// coalesced (16 inputs each), sum the planes in fp32 (smallest first), multiply-add the
-// CTA's tokens and reduce across the warp.  The group statistics are block reductions.
+// this kernel instead: a cluster of kSmallSlices CTAs per (group, 8 tokens), so that the
+// group's 384 KB of R-plane rows are read by eight SMs.  CTA s of a cluster computes
+// output coordinates 128g + 16s .. +15, two per warp: for each, the 32 lanes read the
+// three R-plane rows coalesced (16 inputs each), sum the planes in fp32 (smallest first),
+// multiply-add the CTA's tokens and reduce across the warp; the results go straight into
+// the shared memory of the cluster's first CTA, which computes the group statistics
+// (block reductions) and stores the records.
 constexpr int kSmallTok = 8;
 constexpr int kSmallMaxN = 64;
-constexpr int kSmallThreads = 512;
-constexpr int kSmallOutPerWarp = ROLAQ_GROUP / (kSmallThreads / 32);   // 8
+constexpr int kSmallSlices = 8;
+constexpr int kSmallThreads = 256;
+constexpr int kSmallOutPerCta = ROLAQ_GROUP / kSmallSlices;                  // 16
+constexpr int kSmallOutPerWarp = kSmallOutPerCta / (kSmallThreads / 32);    // 2
 
 __device__ __forceinline__ float block_sum128(float v, float* red) {
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -384,15 +389,16 @@ __device__ __forceinline__ float block_sum128(float v, float* red) {
     return r;
 }
 
-__global__ void __launch_bounds__(kSmallThreads)
+__global__ void __cluster_dims__(kSmallSlices, 1, 1) __launch_bounds__(kSmallThreads)
 rolaq_quantize_small_kernel(const __nv_bfloat16* __restrict__ R_split, const __nv_bfloat16* __restrict__ c,
                             const QuantArgs args) {
     __shared__ __align__(16) __nv_bfloat16 s_c[kSmallTok][ROLAQ_D_C];
     __shared__ float s_y[kSmallTok][ROLAQ_GROUP];
     __shared__ float s_red[4];
     __shared__ uint32_t s_codes[kSmallTok][8];
-    const int g = blockIdx.x;                    // group
-    const int t0 = blockIdx.y * kSmallTok;
+    const uint32_t rank = cluster_ctarank();     // output slice of the group
+    const int g = blockIdx.y;                    // group
+    const int t0 = blockIdx.z * kSmallTok;
     const int nt = min(kSmallTok, args.n - t0);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int e = threadIdx.x; e < kSmallTok * ROLAQ_D_C / 8; e += blockDim.x) {
@@ -403,11 +409,12 @@ rolaq_quantize_small_kernel(const __nv_bfloat16* __restrict__ R_split, const __n
     }
     if (threadIdx.x < kSmallTok * 8) s_codes[threadIdx.x >> 3][threadIdx.x & 7] = 0;
     __syncthreads();
-    // this lane's 16 inputs of every token, as fp32
+    cluster_sync();                              // every CTA of the cluster is running
+    const uint32_t y_first = mapa_shared(smem_u32(&s_y[0][0]), 0);
     const size_t plane = (size_t)ROLAQ_D_C * ROLAQ_D_C;
-#pragma unroll 2
+#pragma unroll
     for (int oo = 0; oo < kSmallOutPerWarp; ++oo) {
-        const int o = kSmallOutPerWarp * warp + oo;
+        const int o = kSmallOutPerCta * (int)rank + kSmallOutPerWarp * warp + oo;
         float rk[16];
 #pragma unroll
         for (int q8 = 0; q8 < 16; ++q8) rk[q8] = 0.f;
@@ -439,10 +446,11 @@ rolaq_quantize_small_kernel(const __nv_bfloat16* __restrict__ R_split, const __n
                 }
             }
             for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if (lane == 0) s_y[t][o] = acc;
+            if (lane == 0) st_cluster_f32(y_first + (uint32_t)(t * ROLAQ_GROUP + o) * 4u, acc);
         }
     }
-    __syncthreads();
+    cluster_sync();                              // the group's y is complete in the first CTA
+    if (rank != 0) return;
     if (threadIdx.x >= ROLAQ_GROUP) return;      // warps 0..3 finish the group
     const int j = threadIdx.x;
     for (int t = 0; t < nt; ++t) {

@@ -174,7 +174,7 @@ int rolaq_quantize_append(const rolaq_cache* cache, const rolaq_layer_params* p,
         a.n = n;
         a.tau = p->tau;
         a.gain = p->gain;
-        dim3 grid(ROLAQ_GROUPS, (n + kSmallTok - 1) / kSmallTok);
+        dim3 grid(kSmallSlices, ROLAQ_GROUPS, (n + kSmallTok - 1) / kSmallTok);
         rolaq_quantize_small_kernel<<<grid, kSmallThreads, 0, (cudaStream_t)stream>>>(
             reinterpret_cast<const __nv_bfloat16*>(R_split_dev), reinterpret_cast<const __nv_bfloat16*>(c_dev), a);
         return launch_status();

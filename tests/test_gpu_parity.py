@@ -104,6 +104,70 @@ def test_quantize_ragged_multi_request_shuffled_pages():
     assert (pool[pt[0, 0], 288 * 0 + 128:O.PAGE_META] == 0xAB).all()
 
 
+@pytest.mark.parametrize("n", [1, 5, 8, 13, 64])
+def test_small_append_token_counts(n):
+    """Calls of up to 64 tokens take the clustered small-append kernel: blocks of 8 tokens
+    with a ragged last block, scattered positions of several requests, sink and recent
+    positions included; every record against the oracle, other rows untouched."""
+    B, cap, n_sink, n_recent = 4, 256, 4, 16
+    w = W.Workload(f"sa{n}", B, (cap,) * B, 16, paged_shuffled=True, seed=500 + n)
+    tau, gain = 0.93, 1.09
+    Rm = W.rotation(w.seed)
+    R_split = R.prepare_rotation(torch.as_tensor(Rm).to(DEV))
+    pt = W.page_table(w)
+    cache = R.PagedCache(int(pt.max()) + 1, torch.as_tensor(pt), n_sink, n_recent, device=DEV)
+    cache.pages.fill_(0xAB)
+    rng = np.random.default_rng(n)
+    flat = rng.choice(B * cap, n, replace=False)
+    flat[0] = 2                                    # a sink position
+    if n > 1:
+        flat[1] = cap + cap - 1                    # a recent position of request 1
+    flat = np.unique(flat)
+    rng.shuffle(flat)
+    req = (flat // cap).astype(np.int32)
+    pos = (flat % cap).astype(np.int32)
+    m = len(flat)
+    c = W.latent(w, 0, m, stream=7)
+    kr = W.rope_key(w, 0, m, stream=8)
+    lens = torch.full((B,), cap, dtype=torch.int32, device=DEV)
+    p = R.layer_params_init(tau, gain)
+    R.quantize_append(cache, p, R_split, c.to(DEV), kr.to(DEV), torch.as_tensor(req).to(DEV),
+                      torch.as_tensor(pos).to(DEV), lens)
+    torch.cuda.synchronize()
+    pool = cache.pages.cpu().numpy()
+    q = O.quantize(f64(c), Rm.astype(np.float64), tau, gain)
+    recs = [O.pages_read(pool, pt, int(b), int(s) + 1, start=int(s)) for b, s in zip(req, pos)]
+    packed = np.stack([x[0][0] for x in recs])
+    meta = np.stack([x[1][0] for x in recs])
+    krb = np.stack([x[2][0] for x in recs])
+    ok, frac, nbad = codes_match(packed, q, tau)
+    assert ok, nbad
+    emu, es = meta_match(meta, q, gain)
+    assert emu <= META_TOL and es <= META_TOL, (emu, es)
+    assert (krb == bf16_bits(kr)).all()
+    prot = cache.prot.float().cpu().numpy().astype(np.float64)
+    seen = 0
+    for t, (b, s) in enumerate(zip(req, pos)):
+        if s < n_sink:
+            slot = s
+        elif s >= cap - n_recent:
+            slot = n_sink + s % n_recent
+        else:
+            continue
+        seen += 1
+        y = q["y"][t]
+        tol = np.abs(y) * 2.0 ** -7 + 1e-5 * np.abs(y).max()
+        assert (np.abs(prot[b, slot] - y) <= tol).all(), (b, s)
+    assert seen >= 1
+    pages = pool.reshape(-1, O.PAGE_BYTES)
+    written = set(zip(req.tolist(), pos.tolist()))
+    for b in range(B):
+        for s in range(0, cap, 7):
+            if (b, s) not in written:
+                row = s % O.PAGE_TOKENS
+                assert (pages[pt[b, s // O.PAGE_TOKENS], row * 128:(row + 1) * 128] == 0xAB).all(), (b, s)
+
+
 def test_quantize_protected_side_store():
     w = W.Workload("prot", 2, (200, 40), 16, seed=78)
     tau, gain = 1.05, 1.12
