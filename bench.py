@@ -276,7 +276,8 @@ def run_ours(args, rank, world, dev):
 
     # prefill write path: 65,536 tokens x 27 layers
     q_stats = bench_quantize(args, dev, world)
-    clocks = sampler.stop()     # sampled across the three timed regions
+    bf16_stats = bench_bf16_baseline(args, dev, world, w, dec_ms)
+    clocks = sampler.stop()     # sampled across the timed regions
 
     hbm, bf16, src = peaks()
     dec_bytes = w.total_tokens * R.TOKEN_BYTES
@@ -300,6 +301,7 @@ def run_ours(args, rank, world, dev):
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": args.steps * w.layers * 3,
         "quantize": q_stats,
+        "bf16_baseline": bf16_stats,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -352,6 +354,55 @@ def bench_quantize(args, dev, world):
                          "executed_flops_factor": 3, "peak_source": src},
             "hbm": {"achieved": round(bytes_ / (per_launch_ms * 1e-3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
                     "frac": round(bytes_ / (per_launch_ms * 1e-3) / 1e9 / hbm, 4)}}
+
+
+# ------------------------------------------------------------- BF16 baseline ----
+# The same decode on an uncompressed cache (1,152 B per token: 512 bf16 latent + 64 bf16
+# RoPE key, 64-token pages), run by a library kernel: FlashInfer's TRT-LLM-generated MLA
+# decode for Blackwell.  It is a comparison point (the pages compare their 2-bit decode
+# with BF16 on the same GPU), never part of this library's path.
+
+def bench_bf16_baseline(args, dev, world, w, dec_ms):
+    try:
+        from flashinfer import mla as fi_mla
+    except Exception as e:                      # library missing: no baseline, say why
+        return {"unavailable": f"flashinfer not importable: {type(e).__name__}"}
+    B, L, H = w.batch, w.seq_lens[0], w.heads
+    page = R.PAGE_TOKENS
+    npg = (L + page - 1) // page
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    kv = torch.randn((B * npg, page, 576), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    bt = torch.arange(B * npg, dtype=torch.int32, device=dev).reshape(B, npg)
+    lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+    q = torch.randn((B, 1, H, 576), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    ws = torch.zeros(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        fi_mla.trtllm_batch_decode_with_kv_cache_mla(q, kv, ws, 128, 512, 64, bt, lens, L,
+                                                    bmm1_scale=SM_SCALE, bmm2_scale=1.0)
+
+    for _ in range(max(args.warmup, 1)):
+        call()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    reps = max(args.steps, 1) * 4
+    t0.record(stream)
+    for _ in range(reps):
+        call()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world) / reps
+    nbytes = B * L * 1152
+    del kv
+    return {"kernel": "flashinfer trtllm_batch_decode_with_kv_cache_mla (library), bf16 cache",
+            "workload": f"{B} x {L} tokens, {H} heads, one layer", "bytes_per_token": 1152,
+            "ms_per_call": round(ms, 4), "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "tokens_per_s": round(B * L / (ms * 1e-3), 1),
+            "time_ratio_bf16_over_2bit": round(ms / dec_ms, 3), "capacity_ratio": 4.0}
 
 
 # ------------------------------------------------------------ profiling cases ----
