@@ -3,30 +3,26 @@
 // softmax over the request's tokens, 512-d latent readout in the rotated basis.
 //
 // Kernel A (rolaq_decode_split): one CTA per (work item, 16-head chunk).  A work item is a
-// run of whole pages of one request (split-K over the sequence).  16 warps in four teams
-// of four; team t takes pages t, t+4, t+8, ... of the item and keeps its own online
-// softmax state, and the four teams are merged inside the CTA at the end, so each item
-// writes one partial.  Lane 0 of a team's first warp streams its pages (one 144-row bulk
-// tensor copy per page, 128-byte swizzle) through two shared-memory stages and issues the
-// team's tensor-core MMAs.  Inside a team, warp q owns content channels 32q..32q+31 of
-// every 128-channel group (the TMEM lane quarter it may access) and RoPE channels
-// 16q..16q+15.
-//
-// A team walks its tokens in steps of 16 with one team barrier per step:
-//   dequant  per (token, group) the four fp16 values mean + scale * level are prepared
-//            one step ahead; a PRMT lookup turns every 2-bit code straight into x (fp16;
-//            bf16 would round all channels sharing a code the same way and cost ~5x in
-//            output error).
-//   QK       mma.sync m16n8k16 (heads = M) on those x fragments in registers; partial
-//            scores of the four warps meet in shared memory.
-//   A tile   the same fragments transposed (movmatrix) and stored to tensor memory with
-//            lanes = channels, columns = tokens (two-slot ring).
-//   softmax  warp q takes heads 4q..4q+3; the running max moves only when a score exceeds
-//            it by more than 2^8 (one warp vote in the common case); probabilities go to
-//            shared memory as the fp16 B operand.
-//   PV       tcgen05.mma M = 128 channels of a group, N = 16 heads, K = 16 tokens, A from
-//            tensor memory, accumulating O (fp32) in tensor memory; a rare rescale pass
-//            multiplies O when a head's running max moves.
+// run of whole pages of one request (split-K over the sequence).  Each 64-token page is
+// one tile, handled by warps with fixed roles and handed on through mbarriers:
+//   warp 0 (lane 0)   streams the pages (one 144-row bulk tensor copy each, 128-byte
+//                     swizzle) through kStages shared-memory stages;
+//   warps 8..15       dequantise: thread (token t, group g) forms the four fp16 values
+//                     mean + scale * level of its (token, group) and turns its 128 codes
+//                     into x with one PRMT per pair, stored straight into a 128-byte-
+//                     swizzled x tile [64 tokens][512 channels] (two tiles, double
+//                     buffered).  fp16, not bf16: channels sharing a code share one
+//                     rounding error, which bf16 makes ~5x too large in the output;
+//   warp 1 (lane 0)   issues the tensor-core MMAs: QK as tcgen05.mma M = 64 tokens,
+//                     N = 16 heads, K = 512 (fp16, A = the x tile) plus K = 64 (bf16,
+//                     A = the staged page's RoPE rows), S in tensor memory; PV as
+//                     tcgen05.mma M = 128 channels of a group, N = 16 heads, K = 64
+//                     tokens, A = the same x tile read transposed (MN-major), B = P,
+//                     O (fp32) accumulated in tensor memory;
+//   warps 4..7        softmax: one tensor-memory load gives a token's 16 scores; the
+//                     running max moves only when a score exceeds it by more than 2^8
+//                     (a vote in the common case), in which case O is rescaled before
+//                     the next PV; P goes to shared memory as the fp16 B operand.
 // Kernel B (rolaq_decode_merge): log-sum-exp merge of the per-item partials.
 #pragma once
 #include "common.cuh"
@@ -35,18 +31,19 @@ namespace rolaq {
 
 constexpr int kPageTok = ROLAQ_PAGE_TOKENS;
 constexpr int kPageRows = ROLAQ_PAGE_BYTES / 128;   // 144 rows of 128 B
-constexpr int kTeams = 4;
-constexpr int kDecodeThreads = 128 * kTeams;
-constexpr int kStages = 2;                          // whole pages in flight per team
-constexpr int kRing = 2;                            // TMEM A slots / P tiles per team
-constexpr int kStepTok = 16;                        // tokens per step
-constexpr int kRingCol = 64;                        // O: columns 0..63 (16 per group)
-constexpr int kTeamCols = kRingCol + 32 * kRing;    // TMEM columns per team (ring after O)
-static_assert(kTeams * kTeamCols <= 512, "tensor memory columns");
-constexpr int kLutStride = 6;                       // uint2 per token row of the LUT tile
-constexpr float kRescaleLog2 = 8.f;
+constexpr int kDecodeThreads = 512;
+constexpr int kStages = 3;                          // pages in flight
+constexpr int kSoftWarp0 = 4;                       // softmax warps 4..7 (TMEM lane quarters)
+constexpr int kDqWarp0 = 8;                         // dequant warps 8..15
+constexpr int kXAtom = kPageTok * 128;              // one 64-channel column block of an x tile
+constexpr int kXTile = 8 * kXAtom;                  // 64 KB: 64 tokens x 512 fp16
 constexpr int kMetaRow = 64;                        // page rows: codes 0..63, meta 64..79,
 constexpr int kKrRow = 80;                          // RoPE keys 80..143
+constexpr int kSCol = 0;                            // TMEM: S tiles at columns 0 and 16
+constexpr int kOCol = 64;                           //       O at 64..127 (16 per group)
+constexpr int kTmemCols = 128;
+constexpr float kRescaleLog2 = 8.f;
+constexpr float kF16Max = 65504.f;
 
 struct DecodeArgs {
     const int32_t* page_table;
@@ -66,16 +63,23 @@ struct DecodeArgs {
 };
 
 struct DecodeSmem {
-    alignas(1024) uint8_t stage[kTeams][kStages][ROLAQ_PAGE_BYTES];
-    float sT[kTeams][2][4][16][16];          // partial scores [team][buf][warp][head][token']
-    alignas(128) uint8_t P[kTeams][kRing][512];   // fp16 probabilities, UMMA B layout
-    alignas(16) uint2 lut[kTeams][2][kStepTok][kLutStride];   // (lo, hi) bytes of 4 x values
-    float sAl[kTeams][2][16];                // rescale factor per head
-    float2 team_ml[kTeams][16];
-    int resc[kTeams][2];
-    alignas(8) uint64_t full[kTeams][kStages];
-    alignas(8) uint64_t pvbar[kTeams][kRing];
-    int valid[kTeams][kStages];
+    alignas(1024) uint8_t x[2][kXTile];                   // x tiles (K-major, 128-byte swizzle)
+    alignas(1024) uint8_t stage[kStages][ROLAQ_PAGE_BYTES];
+    alignas(128) uint8_t qc[16 * ROLAQ_D_C * 2];          // fp16 query, QK B operand
+    alignas(128) uint8_t qr[16 * ROLAQ_D_R * 2];          // bf16 RoPE query, B operand
+    alignas(128) uint8_t P[2][16 * kPageTok * 2];         // fp16 probabilities, PV B operand
+    float red[4][16];                                     // softmax warps: per-warp head values
+    float mref[16];                                       // running reference max per head
+    float alpha[16];                                      // its last rescale factor
+    int vote[2][4];
+    alignas(8) uint64_t full[kStages];     // page copy landed
+    alignas(8) uint64_t pfree[kStages];    // page read by the dequant warps and the QK MMAs
+    alignas(8) uint64_t xready[2];         // x tile written
+    alignas(8) uint64_t xfree[2];          // PV of the tile done (x tile and P buffer free)
+    alignas(8) uint64_t sfull[2];          // QK of the tile done
+    alignas(8) uint64_t sfree[2];          // scores read by the softmax warps
+    alignas(8) uint64_t pready[2];         // P written (and O rescaled if needed)
+    int valid[kStages];
     uint32_t tmem_base;
     int plan[4];
     int abort;
@@ -146,22 +150,6 @@ __device__ PlanInfo plan_lookup(const int32_t* seq_lens, int batch, int target, 
     return pi;
 }
 
-// Instruction descriptor of the PV MMA: f16 x f16 -> f32, M = 128, N = 16.
-constexpr uint32_t kPvIdesc = (1u << 4) | ((16u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr float kF16Max = 65504.f;
-
-// Shared-memory descriptor of a K-major operand without swizzle: 8-row x 16-byte core
-// matrices, K-adjacent cores 128 B apart, 8-row groups 256 B apart.
-__device__ __forceinline__ uint64_t umma_desc_plain(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 16) |
-           ((uint64_t)(256 >> 4) << 32) | (1ull << 46);
-}
-// D (tensor memory) (+)= A (tensor memory) * B (shared memory)
-__device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t acc) {
-    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-                 :: "r"(d), "r"(a), "l"(bdesc), "r"(kPvIdesc), "r"(acc) : "memory");
-}
 // Eight fp16 pairs from one 32-bit word of codes: bytes 0-1 hold 8 codes of token A,
 // bytes 2-3 8 codes of token B (code j of a byte at bits 2j).  r[k][0] = (x_A of code k
 // of byte 0, x_A of code k of byte 1); r[k][1] the same for token B.  A token's lookup
@@ -184,229 +172,142 @@ __device__ __forceinline__ void dequant_word2(uint32_t w, uint2 la, uint2 lb, ui
     r[3][1] = prmt(lb.x, lb.y, __umulhi(m3, 0x11u << 10) + 0x4040u);
 }
 
+// ---- tensor-core operands -----------------------------------------------------
+// Shared-memory matrix descriptor (sm_100 form): start, leading / stride byte offsets
+// (16-byte units), version 1, layout type (0: no swizzle, 2: 128-byte swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+// Instruction descriptors: fp32 accumulate, K-major unless noted, N = 16 heads.
+constexpr uint32_t kIdQk = (1u << 4) | ((16u >> 3) << 17) | ((64u >> 4) << 24);                 // f16, M = 64
+constexpr uint32_t kIdRope = kIdQk | (1u << 7) | (1u << 10);                                     // bf16, M = 64
+constexpr uint32_t kIdPv = (1u << 4) | (1u << 15) | ((16u >> 3) << 17) | ((128u >> 4) << 24);   // f16, M = 128, A MN-major
+
+// D (tensor memory) (+)= A (shared memory) * B (shared memory).  Called by a whole warp
+// with warp-uniform operands (so they live in uniform registers); one elected lane issues.
+__device__ __forceinline__ void umma_ss(uint32_t d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+    asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d), "l"(da), "l"(db), "r"(idesc), "r"(acc) : "memory");
+}
+// One lane of a converged warp (elect.sync).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t p;
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\tselp.u32 %0, 1, 0, e;\n\t}" : "=r"(p));
+    return p != 0;
+}
+// Single-thread forms, for a batch issued inside one elected branch.
+__device__ __forceinline__ void umma_ss1(uint32_t d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d), "l"(da), "l"(db), "r"(idesc), "r"(acc) : "memory");
+}
+// tcgen05.commit from one elected lane of a converged warp.
+__device__ __forceinline__ void umma_commit_warp(uint32_t bar) {
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+                 :: "r"(bar) : "memory");
+}
+
+// Column slot of channel order inside every 16-channel block: the PRMT lookup yields the
+// pairs (k, k+4), so slot 2k + e of a block of 8 holds channel k + 4e.  The query is laid
+// out in slot order and O rows come back in slot order; this maps a slot to its channel.
+__host__ __device__ __forceinline__ int slot_channel(int s) {
+    return (s & ~7) + ((s & 7) >> 1) + 4 * (s & 1);
+}
+// Byte offset of (row, 16-byte chunk) in an x tile: 64-channel column blocks of
+// [64 rows][128 B], chunks XOR row % 8 (the tensor cores' 128-byte swizzle).
+__device__ __forceinline__ uint32_t x_off(int row, int chunk) {
+    return (chunk >> 3) * kXAtom + row * 128 + ((((chunk & 7) ^ row) & 7) << 4);
+}
+// K-major operand without swizzle (8-row x 16-byte core matrices, K-adjacent cores 128 B
+// apart, 8-row groups `sbo` apart): byte offset of element (row n, k), 2-byte elements.
+__device__ __forceinline__ uint32_t plain_off(int n, int k, int sbo) {
+    return (n >> 3) * sbo + (k >> 3) * 128 + (n & 7) * 16 + (k & 7) * 2;
+}
+
+// Page-table entry of page `page_idx` of request b (-1 past the table).
+__device__ __forceinline__ long long page_id(const DecodeArgs& args, int b, int page_idx) {
+    return page_idx < args.max_pages ? (long long)args.page_table[(long long)b * args.max_pages + page_idx] : -1;
+}
+__device__ __forceinline__ bool page_ok(const DecodeArgs& args, long long pid) {
+    return pid >= 0 && pid < args.num_pages;
+}
 // Issue the bulk copy of one page (all 144 rows) into stage k % kStages, or mark the
 // stage invalid when the page-table entry is outside the pool.
 __device__ __forceinline__ void load_page(DecodeSmem& sm, const CUtensorMap* map, const DecodeArgs& args,
-                                          int team, int b, int page_idx, int k) {
+                                          long long pid, int k) {
     const int st = k % kStages;
-    long long pid = -1;
-    if (page_idx < args.max_pages) pid = args.page_table[(long long)b * args.max_pages + page_idx];
-    const uint32_t bar = smem_u32(&sm.full[team][st]);
-    if (pid >= 0 && pid < args.num_pages) {
-        sm.valid[team][st] = 1;
+    const uint32_t bar = smem_u32(&sm.full[st]);
+    if (page_ok(args, pid)) {
+        sm.valid[st] = 1;
         mbar_arrive_expect_tx(bar, ROLAQ_PAGE_BYTES);
-        tma_load_2d(smem_u32(sm.stage[team][st]), map, 0, (int)(pid * kPageRows), bar);
+        tma_load_2d(smem_u32(sm.stage[st]), map, 0, (int)(pid * kPageRows), bar);
     } else {
-        sm.valid[team][st] = 0;
+        sm.valid[st] = 0;
         raise_status(ROLAQ_STATUS_BAD_PAGE);
         mbar_arrive(bar);
     }
 }
 
-// Lookup pair of token tt (0..15 of step `sub` of a staged page), group gg: fp16 of
-// mean + scale * (-b, -a, a, b), split into low bytes and high bytes.  Tokens past the
-// sequence end or on an invalid page get zeros, so their x is 0 (their scores are masked).
-// Values beyond the fp16 range raise ROLAQ_STATUS_RANGE.
-__device__ __forceinline__ void lut_prep(const uint8_t* pg, bool vpage, int sub, int tt, int gg, int pos,
-                                         int L, float la, float lb, uint2* lut) {
-    uint2 v = make_uint2(0u, 0u);
-    if (vpage && pos < L) {
-        const int pt = kStepTok * sub + tt;
-        const float2 ms = *reinterpret_cast<const float2*>(
-            pg + swz128(kMetaRow + (pt >> 2), (pt & 3) * 32 + 8 * gg));
+// One dequant thread's share of a tile: token row t, channel group g.  The four fp16
+// values mean + scale * (-b, -a, a, b) are split into low and high bytes so that a PRMT
+// picks value c with nibbles c and c + 4; each 32-bit word of codes (16 channels) gives
+// eight fp16 pairs (o[w][0..3] and o[w][4..7]: two 16-byte chunks of the x tile in slot
+// order).  Tokens past the sequence end (or on an invalid page) get x = 0; protected
+// tokens take their bf16 side-store row instead of the codes.  Computed into registers
+// before the x buffer is free, stored after.
+__device__ __forceinline__ void dequant_tile_part(const uint8_t* pg, int t, int g, bool valid, bool prot,
+                                                  const __nv_bfloat16* prow, float la, float lb,
+                                                  uint32_t (&o)[8][8]) {
+    uint2 lut = make_uint2(0u, 0u);
+    uint4 cw0 = make_uint4(0u, 0u, 0u, 0u), cw1 = cw0;
+    if (valid) {
+        const float2 ms = *reinterpret_cast<const float2*>(pg + swz128(kMetaRow + (t >> 2), (t & 3) * 32 + 8 * g));
         if (!(fabsf(ms.x) + fabsf(ms.y) * lb < kF16Max)) raise_status(ROLAQ_STATUS_RANGE);
         const uint32_t w01 = pack_f16(fmaf(ms.y, -lb, ms.x), fmaf(ms.y, -la, ms.x));
         const uint32_t w23 = pack_f16(fmaf(ms.y, la, ms.x), fmaf(ms.y, lb, ms.x));
-        v.x = prmt(w01, w23, 0x6420u);
-        v.y = prmt(w01, w23, 0x7531u);
+        lut.x = prmt(w01, w23, 0x6420u);
+        lut.y = prmt(w01, w23, 0x7531u);
+        cw0 = *reinterpret_cast<const uint4*>(pg + t * 128 + (((2 * g) ^ (t & 7)) << 4));
+        cw1 = *reinterpret_cast<const uint4*>(pg + t * 128 + (((2 * g + 1) ^ (t & 7)) << 4));
     }
-    lut[tt * kLutStride + gg] = v;
-}
-
-// Per-thread byte offsets inside a staged page, fixed for the whole kernel: every step's
-// code and RoPE rows start at a multiple of 8, so the 128-byte swizzle of a thread's
-// position does not depend on the step (step sub adds 2048, the second n-tile 1024).
-struct StageOffsets {
-    uint32_t code[4];      // codes of token r, channels 32q + 8i.. of group g
-    uint32_t kr0, kr1;     // RoPE channels 16q + 2i.. and 16q + 8 + 2i.. of token r
-};
-__device__ __forceinline__ StageOffsets stage_offsets(int q, int r, int i) {
-    StageOffsets o;
+    const uint32_t cw[8] = {cw0.x, cw0.y, cw0.z, cw0.w, cw1.x, cw1.y, cw1.z, cw1.w};
 #pragma unroll
-    for (int g = 0; g < 4; ++g)
-        o.code[g] = r * 128 + (((2 * g + (q >> 1)) ^ r) << 4) + ((8 * q + 2 * i) & 15);
-    o.kr0 = (kKrRow + r) * 128 + (((2 * q) ^ r) << 4) + 4 * i;
-    o.kr1 = (kKrRow + r) * 128 + (((2 * q + 1) ^ r) << 4) + 4 * i;
-    return o;
-}
-
-// QK of one 16-token step for warp q, one channel group at a time.  Thread (r, i) builds
-// the x fragments of tokens r and r + 8 for channels 32q + 8i .. 32q + 8i + 7 of group g:
-// x[ks][nt][h] holds B-fragment k indices 2i + 8h + {0,1} of k-slice ks, which are
-// channels 32q + 8i + 2ks + h + {0, 4} (the query fragments use the same order).  Right
-// after its MMAs each group's fragments are transposed and stored as the PV A operand
-// (lanes 32q + 16ks + y for B-fragment k index y; ring columns 8g + c, where column 2i
-// holds tokens (2i, 2i+1) and column 2i + 1 tokens (8 + 2i, 9 + 2i)); the ring slot is
-// waited for before the first store.  Scores of the 16 heads x 16 tokens over this warp's
-// channels (plus its RoPE channels) go to sT with the token index XOR 8 * ((head >> 1) & 1)
-// (conflict-free stores and loads).  `pg` points at the step's first row.  PROT: some
-// token of the step is protected and takes its x from the bf16 side store (as fp16).
-template <bool PROT>
-__device__ __forceinline__ void qk_step(const uint8_t* pg, const StageOffsets& so, const uint2* lut,
-                                        float (*sT)[16], int q, int r, int i, const uint32_t (&qa)[4][2][4],
-                                        const uint32_t (&qra)[4], uint32_t a_taddr, uint32_t slot_bar,
-                                        unsigned slot_parity, bool slot_wait, volatile int* abort, int pos0,
-                                        int L, int recent_start, const DecodeArgs& args, int b) {
-    bool pa = false, pb = false;
-    const uint4* srca = nullptr;
-    const uint4* srcb = nullptr;
-    if (PROT) {
-        const int nslot = args.n_sink + args.n_recent;
-        const int p0 = pos0 + r, p1 = pos0 + 8 + r;
-        pa = p0 < L && (p0 < args.n_sink || p0 >= recent_start);
-        pb = p1 < L && (p1 < args.n_sink || p1 >= recent_start);
-        const int s0 = p0 < args.n_sink ? p0 : args.n_sink + p0 % max(args.n_recent, 1);
-        const int s1 = p1 < args.n_sink ? p1 : args.n_sink + p1 % max(args.n_recent, 1);
-        srca = reinterpret_cast<const uint4*>(args.prot + ((size_t)b * nslot + s0) * ROLAQ_D_C + 32 * q + 8 * i);
-        srcb = reinterpret_cast<const uint4*>(args.prot + ((size_t)b * nslot + s1) * ROLAQ_D_C + 32 * q + 8 * i);
+    for (int w = 0; w < 8; ++w) {
+        uint32_t r[4][2];
+        dequant_word2(cw[w], lut, lut, r);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) { o[w][k] = r[k][0]; o[w][4 + k] = r[k][1]; }
     }
-    float acc[2][4];
+    if (prot) {
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+        for (int w = 0; w < 8; ++w) {
+            // channels 128g + 16w + {0..15} from the side store, in slot order
+            const uint4 u0 = reinterpret_cast<const uint4*>(prow + 128 * g + 16 * w)[0];
+            const uint4 u1 = reinterpret_cast<const uint4*>(prow + 128 * g + 16 * w)[1];
+            const uint32_t v[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) {
-        const uint32_t c0 = *reinterpret_cast<const uint16_t*>(pg + so.code[g]);
-        const uint32_t c1 = *reinterpret_cast<const uint16_t*>(pg + so.code[g] + 1024);
-        uint32_t t[4][2];
-        dequant_word2(c0 | (c1 << 16), lut[r * kLutStride + g], lut[(r + 8) * kLutStride + g], t);
-        uint32_t x[2][2][2];
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) x[ks][nt][h] = t[2 * ks + h][nt];
-        if (PROT) {
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                if (nt == 0 ? pa : pb) {
-                    const uint4 u = (nt == 0 ? srca : srcb)[16 * g];
-                    x[0][nt][0] = pack_f16(bf16_lo(u.x), bf16_lo(u.z));
-                    x[0][nt][1] = pack_f16(bf16_hi(u.x), bf16_hi(u.z));
-                    x[1][nt][0] = pack_f16(bf16_lo(u.y), bf16_lo(u.w));
-                    x[1][nt][1] = pack_f16(bf16_hi(u.y), bf16_hi(u.w));
-                }
+            for (int k = 0; k < 4; ++k) {
+                // slot pair k of each 8-block: channels (k, k + 4) of the block
+                const float a0 = (k & 1) ? bf16_hi(v[k >> 1]) : bf16_lo(v[k >> 1]);
+                const float a1 = (k & 1) ? bf16_hi(v[2 + (k >> 1)]) : bf16_lo(v[2 + (k >> 1)]);
+                const float b0 = (k & 1) ? bf16_hi(v[4 + (k >> 1)]) : bf16_lo(v[4 + (k >> 1)]);
+                const float b1 = (k & 1) ? bf16_hi(v[6 + (k >> 1)]) : bf16_lo(v[6 + (k >> 1)]);
+                o[w][k] = pack_f16(a0, a1);
+                o[w][4 + k] = pack_f16(b0, b1);
             }
         }
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) mma_f16_16816(acc[nt], qa[g][ks], x[ks][nt][0], x[ks][nt][1]);
-        if (g == 0) {
-            if (slot_wait) mbar_wait(slot_bar, slot_parity, abort);
-            tc_fence_after();
-        }
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-            const uint32_t v0 = movmatrix_trans(x[ks][0][0]);
-            const uint32_t v1 = movmatrix_trans(x[ks][1][0]);
-            const uint32_t v2 = movmatrix_trans(x[ks][0][1]);
-            const uint32_t v3 = movmatrix_trans(x[ks][1][1]);
-            asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1, %2, %3, %4};"
-                         :: "r"(a_taddr + ((uint32_t)(16 * ks) << 16) + 8 * g), "r"(v0), "r"(v1), "r"(v2),
-                            "r"(v3)
-                         : "memory");
-        }
-    }
-    const int sw = 8 * ((r >> 1) & 1);
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-        // RoPE part of the score for channels 16q..16q+15
-        const uint32_t kb0 = *reinterpret_cast<const uint32_t*>(pg + so.kr0 + 1024 * nt);
-        const uint32_t kb1 = *reinterpret_cast<const uint32_t*>(pg + so.kr1 + 1024 * nt);
-        mma_bf16_16816(acc[nt], qra, kb0, kb1);
-        const int t = (8 * nt + 2 * i) ^ sw;
-        *reinterpret_cast<float2*>(&sT[r][t]) = make_float2(acc[nt][0], acc[nt][1]);
-        *reinterpret_cast<float2*>(&sT[r + 8][t]) = make_float2(acc[nt][2], acc[nt][3]);
     }
 }
-
-// Softmax of one step for head hh (of the 16-head chunk), tokens 2jj, 2jj+1.  The
-// reference max m_ref moves only when a score exceeds it by more than kRescaleLog2
-// (one warp vote in the common case), so probabilities relative to m_ref stay below
-// 2^kRescaleLog2.  The fp16 probabilities go to the B tile at K positions
-// 4jj, 4jj+1 (jj < 4) or 4(jj-4)+2, +3, matching the A tile's column order.
-__device__ __forceinline__ void softmax_step(const float (*sT)[16][16], uint8_t* Pt, float* sAl, int* resc,
-                                             int hh, int jj, int nvalid, float scale_log2, bool first,
-                                             float& m_ref, float& l_part) {
-    const int t = (2 * jj) ^ (8 * ((hh >> 1) & 1));
-    const float2 v0 = *reinterpret_cast<const float2*>(&sT[0][hh][t]);
-    const float2 v1 = *reinterpret_cast<const float2*>(&sT[1][hh][t]);
-    const float2 v2 = *reinterpret_cast<const float2*>(&sT[2][hh][t]);
-    const float2 v3 = *reinterpret_cast<const float2*>(&sT[3][hh][t]);
-    float s0 = ((v0.x + v1.x) + (v2.x + v3.x)) * scale_log2;
-    float s1 = ((v0.y + v1.y) + (v2.y + v3.y)) * scale_log2;
-    if (2 * jj >= nvalid) s0 = -INFINITY;
-    if (2 * jj + 1 >= nvalid) s1 = -INFINITY;
-    float alpha = 1.f;
-    const bool up = fmaxf(s0, s1) > m_ref + kRescaleLog2 || (m_ref == -INFINITY && fmaxf(s0, s1) > -INFINITY);
-    if (__any_sync(0xffffffffu, up)) {
-        float pm = fmaxf(s0, s1);
-        pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 1));
-        pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 2));
-        pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, 4));
-        if (pm > m_ref + kRescaleLog2 || (m_ref == -INFINITY && pm > -INFINITY)) {
-            alpha = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - pm);
-            m_ref = pm;
-            l_part *= alpha;
-        }
-    }
-    const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-    const float p0 = ex2(s0 - mu), p1 = ex2(s1 - mu);
-    l_part += p0 + p1;
-    const int kp = jj < 4 ? 4 * jj : 4 * (jj - 4) + 2;
-    const int off = (hh >> 3) * 256 + (kp >> 3) * 128 + (hh & 7) * 16 + (kp & 7) * 2;
-    *reinterpret_cast<uint32_t*>(Pt + off) = pack_f16(p0, p1);
-    if (jj == 0) sAl[hh] = alpha;
-    if (alpha != 1.f && !first) *resc = 1;
-}
-
-// PV of team step jp, called by all 128 threads of the team after the step barrier that
-// follows softmax(jp).  When some head's running max moved at jp, every warp first scales
-// its lanes of O (the PV of step jp-1 has completed: its ring slot was waited for), then
-// lane 0 of the team's first warp issues the four group MMAs and commits them to the
-// slot's barrier.
-__device__ __forceinline__ void pv_issue(DecodeSmem& sm, int team, int q, int lane, int jp, uint32_t tmem,
-                                         int bar_id) {
-    const int buf = jp & 1;
-    if (sm.resc[team][buf]) {
-        tc_fence_after();
-        const uint32_t ocol = tmem + ((uint32_t)(32 * q) << 16) + team * kTeamCols;
-#pragma unroll 1
-        for (int g = 0; g < 4; ++g) {
-            uint32_t u[16];
-            tmem_ld16(ocol + 16 * g, u);
-            tmem_ld_wait();
+__device__ __forceinline__ void store_tile_part(uint8_t* xt, int t, int g, const uint32_t (&o)[8][8]) {
 #pragma unroll
-            for (int h = 0; h < 16; ++h) u[h] = __float_as_uint(__uint_as_float(u[h]) * sm.sAl[team][buf][h]);
-            tmem_st16(ocol + 16 * g, u);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        named_bar_sync(bar_id, 128);
-        if (q == 0 && lane == 0) sm.resc[team][buf] = 0;
-    }
-    if (q == 0 && lane == 0) {
-        tc_fence_after();
-        const int slot = jp % kRing;
-        const uint32_t obase = tmem + team * kTeamCols;
-        const uint32_t abase = obase + kRingCol + 32 * slot;
-        const uint64_t bd = umma_desc_plain(smem_u32(sm.P[team][slot]));
-#pragma unroll
-        for (int g = 0; g < 4; ++g) umma_ts(obase + 16 * g, abase + 8 * g, bd, jp > 0 ? 1u : 0u);
-        umma_commit(smem_u32(&sm.pvbar[team][slot]));
+    for (int w = 0; w < 8; ++w) {
+        const int chunk = 16 * g + 2 * w;          // 16-byte chunk index along the 512 slots
+        *reinterpret_cast<uint4*>(xt + x_off(t, chunk)) = make_uint4(o[w][0], o[w][1], o[w][2], o[w][3]);
+        *reinterpret_cast<uint4*>(xt + x_off(t, chunk + 1)) = make_uint4(o[w][4], o[w][5], o[w][6], o[w][7]);
     }
 }
 
@@ -428,11 +329,18 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
         }
     }
     if (threadIdx.x == 32) {
-        for (int t = 0; t < kTeams; ++t) {
-            for (int s = 0; s < kStages; ++s) mbar_init(smem_u32(&sm.full[t][s]), 1);
-            for (int s = 0; s < kRing; ++s) mbar_init(smem_u32(&sm.pvbar[t][s]), 1);
-            sm.resc[t][0] = sm.resc[t][1] = 0;
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_u32(&sm.full[s]), 1);
+            mbar_init(smem_u32(&sm.pfree[s]), (kDecodeThreads / 32 - kDqWarp0) + 1);
         }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&sm.xready[s]), kDecodeThreads / 32 - kDqWarp0);
+            mbar_init(smem_u32(&sm.xfree[s]), 1);
+            mbar_init(smem_u32(&sm.sfull[s]), 1);
+            mbar_init(smem_u32(&sm.sfree[s]), 4);
+            mbar_init(smem_u32(&sm.pready[s]), 4);
+        }
+        for (int h = 0; h < 16; ++h) sm.mref[h] = -INFINITY;
         sm.abort = 0;
         fence_mbar_init();
         prefetch_tmap(&map_page);
@@ -440,188 +348,283 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
     __syncthreads();
     const int b = sm.plan[0];
     if (b < 0) return;                         // item past the end of the plan
-    const int first_page = sm.plan[1], n_pages = sm.plan[2];
+    const int first_page = sm.plan[1], T = sm.plan[2];
     const int L = args.seq_lens[b];
-    const int team = warp >> 2, q = warp & 3;
-    const int tid = threadIdx.x & 127;
-    const bool leader = (q == 0) && (lane == 0);
-    const int n_team = n_pages > team ? (n_pages - team + kTeams - 1) / kTeams : 0;
-    const int J = n_team * (kPageTok / kStepTok);
-    auto page_of = [&](int k) { return first_page + team + kTeams * k; };
-    if (leader)
-        for (int k = 0; k < n_team && k < kStages; ++k) load_page(sm, &map_page, args, team, b, page_of(k), k);
+    const int h0 = hc * 16;
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;"
-                     :: "r"(smem_u32(&sm.tmem_base)) : "memory");
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(&sm.tmem_base)), "r"(kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-
-    const int r = lane >> 2, i = lane & 3;     // mma fragment row group / thread in group
-    const int h0 = hc * 16;
-    // Query fragments (fp16) in the channel order of qk_step.
-    uint32_t qa[4][2][4];
+    // queries as B operands: fp16 content query in slot order, bf16 RoPE query
     {
-        const uint16_t* u0 = reinterpret_cast<const uint16_t*>(args.q + ((size_t)b * args.heads + h0 + r) * ROLAQ_D_C);
-        const uint16_t* u1 = u0 + 8 * ROLAQ_D_C;
+        const uint16_t* qb = reinterpret_cast<const uint16_t*>(args.q + ((size_t)b * args.heads + h0) * ROLAQ_D_C);
         float qmax = 0.f;
-        auto f = [&](const uint16_t* u, int c) {
-            const float v = __uint_as_float((uint32_t)u[c] << 16);
-            qmax = fmaxf(qmax, fabsf(v));
-            return v;
-        };
-#pragma unroll
-        for (int g = 0; g < 4; ++g)
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-                const int c = 128 * g + 32 * q + 8 * i + 2 * ks;
-                qa[g][ks][0] = pack_f16(f(u0, c), f(u0, c + 4));
-                qa[g][ks][1] = pack_f16(f(u1, c), f(u1, c + 4));
-                qa[g][ks][2] = pack_f16(f(u0, c + 1), f(u0, c + 5));
-                qa[g][ks][3] = pack_f16(f(u1, c + 1), f(u1, c + 5));
-            }
+        for (int e = threadIdx.x; e < 16 * ROLAQ_D_C / 2; e += kDecodeThreads) {
+            const int n = e / (ROLAQ_D_C / 2), s = 2 * (e % (ROLAQ_D_C / 2));
+            const float v0 = __uint_as_float((uint32_t)qb[n * ROLAQ_D_C + slot_channel(s)] << 16);
+            const float v1 = __uint_as_float((uint32_t)qb[n * ROLAQ_D_C + slot_channel(s + 1)] << 16);
+            qmax = fmaxf(qmax, fmaxf(fabsf(v0), fabsf(v1)));
+            *reinterpret_cast<uint32_t*>(sm.qc + plain_off(n, s, 64 * 128)) = pack_f16(v0, v1);
+        }
         if (!(qmax < kF16Max)) raise_status(ROLAQ_STATUS_RANGE);
+        const uint32_t* rb = reinterpret_cast<const uint32_t*>(args.qr + ((size_t)b * args.heads + h0) * ROLAQ_D_R);
+        for (int e = threadIdx.x; e < 16 * ROLAQ_D_R / 2; e += kDecodeThreads) {
+            const int n = e / (ROLAQ_D_R / 2), k = 2 * (e % (ROLAQ_D_R / 2));
+            *reinterpret_cast<uint32_t*>(sm.qr + plain_off(n, k, 8 * 128)) = rb[e];
+        }
     }
-    uint32_t qra[4];
-    {
-        const uint32_t* r0 = reinterpret_cast<const uint32_t*>(
-            args.qr + ((size_t)b * args.heads + h0 + r) * ROLAQ_D_R + 16 * q);
-        const uint32_t* r1 = r0 + 8 * ROLAQ_D_R / 2;
-        qra[0] = r0[i];
-        qra[1] = r1[i];
-        qra[2] = r0[4 + i];
-        qra[3] = r1[4 + i];
-    }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    auto page_of = [&](int k) { return first_page + k; };
 
-    const int hh = 4 * q + (lane >> 3), jj = lane & 7;   // softmax: head, token pair
-    const int bar_id = 1 + team;
-    const bool protect = args.n_sink > 0 || args.n_recent > 0;
-    const int recent_start = L - args.n_recent;
-    const float lva = args.level_a, lvb = args.level_b;
-    const uint32_t a_lane = tmem + ((uint32_t)(32 * q) << 16) + team * kTeamCols + kRingCol;
-    const StageOffsets so = stage_offsets(q, r, i);
-    float m_ref = -INFINITY, l_part = 0.f;
-
-    if (J > 0 && tid < 64) {
-        mbar_wait(smem_u32(&sm.full[team][0]), 0, &sm.abort);
-        lut_prep(sm.stage[team][0], sm.valid[team][0] != 0, 0, tid >> 2, tid & 3,
-                 page_of(0) * kPageTok + (tid >> 2), L, lva, lvb, &sm.lut[team][0][0][0]);
-    }
-    named_bar_sync(bar_id, 128);
-
-    for (int j = 0; j < J; ++j) {
-        const int k = j >> 2, sub = j & 3, st = k % kStages;
-        if (sub == 0) mbar_wait(smem_u32(&sm.full[team][st]), (k / kStages) & 1, &sm.abort);
-        const uint8_t* pg = sm.stage[team][st];
-        const int pos0 = page_of(k) * kPageTok + kStepTok * sub;
-        const int nvalid = sm.valid[team][st] ? min(max(L - pos0, 0), kStepTok) : 0;
-        const bool prot = protect && (pos0 < args.n_sink || pos0 + kStepTok > recent_start);
-        const int slot = j % kRing;
-        const uint32_t slot_bar = smem_u32(&sm.pvbar[team][slot]);
-        const unsigned slot_par = (unsigned)(((j - kRing) / kRing) & 1);
-        const uint8_t* pgs = pg + sub * (kStepTok * 128);
-        // QK of step j; its A tile goes to ring slot j % kRing once PV(j - kRing) has read it
-        if (prot)
-            qk_step<true>(pgs, so, &sm.lut[team][j & 1][0][0], sm.sT[team][j & 1][q], q, r, i, qa, qra,
-                          a_lane + 32 * slot, slot_bar, slot_par, j >= kRing, &sm.abort, pos0, L, recent_start,
-                          args, b);
-        else
-            qk_step<false>(pgs, so, &sm.lut[team][j & 1][0][0], sm.sT[team][j & 1][q], q, r, i, qa, qra,
-                           a_lane + 32 * slot, slot_bar, slot_par, j >= kRing, &sm.abort, pos0, L, recent_start,
-                           args, b);
-        tmem_st_wait();
-        tc_fence_before();
-        // lookup pairs of step j + 1
-        if (j + 1 < J && tid < 64) {
-            const int jn = j + 1, kn = jn >> 2, subn = jn & 3, stn = kn % kStages;
-            if (subn == 0) mbar_wait(smem_u32(&sm.full[team][stn]), (kn / kStages) & 1, &sm.abort);
-            lut_prep(sm.stage[team][stn], sm.valid[team][stn] != 0, subn, tid >> 2, tid & 3,
-                     page_of(kn) * kPageTok + kStepTok * subn + (tid >> 2), L, lva, lvb,
-                     &sm.lut[team][jn & 1][0][0]);
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer ----
+        if (lane == 0)
+            for (int k = 0; k < T; ++k) {
+                const int st = k % kStages;
+                if (k >= kStages)
+                    mbar_wait(smem_u32(&sm.pfree[st]), (unsigned)((k / kStages - 1) & 1), &sm.abort);
+                load_page(sm, &map_page, args, page_id(args, b, page_of(k)), k);
+            }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMAs ----
+        // The whole warp runs this loop (warp-uniform descriptors); each MMA and commit is
+        // issued by one elected lane.
+        {
+            // Descriptors are built once; an MMA adds a compile-time byte offset / 16 to the
+            // start-address field (shared addresses stay below 256 KB, so it never carries).
+            const uint64_t dqc = smem_desc(smem_u32(sm.qc), 128, 64 * 128, 0);
+            const uint64_t dqr = smem_desc(smem_u32(sm.qr), 128, 8 * 128, 0);
+            // (buffers of one kind are contiguous: buffer n starts n * size bytes later)
+            const uint64_t dxk = smem_desc(smem_u32(sm.x[0]), 16, 1024, 2);          // K-major view (QK)
+            const uint64_t dxm = smem_desc(smem_u32(sm.x[0]), kXAtom, 1024, 2);      // MN-major view (PV)
+            const uint64_t dp = smem_desc(smem_u32(sm.P[0]), 128, 1024, 0);
+            const uint64_t dkr = smem_desc(smem_u32(sm.stage[0]) + kKrRow * 128, 16, 1024, 2);
+            auto pv = [&](int j) {
+                const int bj = j & 1;
+                mbar_wait(smem_u32(&sm.pready[bj]), (unsigned)((j >> 1) & 1), &sm.abort);
+                __syncwarp();
+                tc_fence_after();
+                const uint64_t da = dxm + (uint64_t)(bj * (kXTile >> 4)), db = dp + (uint64_t)(bj * (sizeof(sm.P[0]) >> 4));
+                const uint32_t first = j > 0 ? 1u : 0u;
+                if (elect_one()) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+#pragma unroll
+                        for (int ks = 0; ks < kPageTok / 16; ++ks)
+                            umma_ss1(tmem + kOCol + 16 * g, da + (uint64_t)((2 * g * kXAtom + ks * 2048) >> 4),
+                                     db + (uint64_t)((ks * 256) >> 4), kIdPv, ks > 0 ? 1u : first);
+                    umma_commit(smem_u32(&sm.xfree[bj]));
+                }
+                __syncwarp();
+            };
+            for (int i = 0; i < T; ++i) {
+                const int bi = i & 1, st = i % kStages;
+                mbar_wait(smem_u32(&sm.xready[bi]), (unsigned)((i >> 1) & 1), &sm.abort);
+                if (i >= 2) mbar_wait(smem_u32(&sm.sfree[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
+                __syncwarp();
+                tc_fence_after();
+                const uint64_t da = dxk + (uint64_t)(bi * (kXTile >> 4));
+                const uint64_t dk = dkr + (uint64_t)(st * (ROLAQ_PAGE_BYTES >> 4));
+                const uint32_t d = tmem + kSCol + 16 * bi;
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < ROLAQ_D_C / 16; ++kk)
+                        umma_ss1(d, da + (uint64_t)(((kk >> 2) * kXAtom + (kk & 3) * 32) >> 4),
+                                 dqc + (uint64_t)((kk * 256) >> 4), kIdQk, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < ROLAQ_D_R / 16; ++kk)
+                        umma_ss1(d, dk + (uint64_t)((kk * 32) >> 4), dqr + (uint64_t)((kk * 256) >> 4), kIdRope, 1u);
+                    umma_commit(smem_u32(&sm.sfull[bi]));
+                    umma_commit(smem_u32(&sm.pfree[st]));
+                }
+                __syncwarp();
+                if (i >= 1) pv(i - 1);
+            }
+            if (T > 0) pv(T - 1);
         }
-        named_bar_sync(bar_id, 128);
-        // page k is fully read after its last step: refill its stage
-        if (leader && sub == 3 && k + kStages < n_team)
-            load_page(sm, &map_page, args, team, b, page_of(k + kStages), k + kStages);
-        if (j >= 1) pv_issue(sm, team, q, lane, j - 1, tmem, bar_id);
-        softmax_step(sm.sT[team][j & 1], sm.P[team][slot], sm.sAl[team][j & 1], &sm.resc[team][j & 1], hh, jj,
-                     nvalid, args.scale_log2, j == 0, m_ref, l_part);
-        fence_proxy_async_smem();
-    }
-    if (J > 0) {
-        if (J >= kRing) mbar_wait(smem_u32(&sm.pvbar[team][J % kRing]), ((J - kRing) / kRing) & 1, &sm.abort);
-        named_bar_sync(bar_id, 128);
-        pv_issue(sm, team, q, lane, J - 1, tmem, bar_id);
-        mbar_wait(smem_u32(&sm.pvbar[team][(J - 1) % kRing]), ((J - 1) / kRing) & 1, &sm.abort);
+    } else if (warp >= kDqWarp0) {
+        // ------------------------------------------------------------- dequant ----
+        const int t = 8 * (warp - kDqWarp0) + (lane & 7), g = lane >> 3;
+        const bool protect = args.n_sink > 0 || args.n_recent > 0;
+        const int nslot = args.n_sink + args.n_recent;
+        const float la = args.level_a, lb = args.level_b;
+        for (int i = 0; i < T; ++i) {
+            const int bi = i & 1, st = i % kStages;
+            mbar_wait(smem_u32(&sm.full[st]), (unsigned)((i / kStages) & 1), &sm.abort);
+            const int pos = page_of(i) * kPageTok + t;
+            const bool valid = sm.valid[st] && pos < L;
+            const bool prot = valid && protect && (pos < args.n_sink || pos >= L - args.n_recent);
+            const __nv_bfloat16* prow = nullptr;
+            if (prot) {
+                const int slot = pos < args.n_sink ? pos : args.n_sink + pos % args.n_recent;
+                prow = args.prot + ((size_t)b * nslot + slot) * ROLAQ_D_C;
+            }
+            uint32_t o[8][8];
+            dequant_tile_part(sm.stage[st], t, g, valid, prot, prow, la, lb, o);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.pfree[st]));      // this warp is done with the page
+            if (i >= 2) mbar_wait(smem_u32(&sm.xfree[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
+            store_tile_part(sm.x[bi], t, g, o);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.xready[bi]));
+        }
+    } else if (warp >= kSoftWarp0) {
+        // ------------------------------------------------------------- softmax ----
+        // Warp q reads TMEM lane quarter q: S rows 16q..16q+15 (M = 64) in lanes 0..15 with
+        // the 16x256b shape, so lane (r, i) holds rows 16q + r and 16q + r + 8 of heads
+        // 2i, 2i+1, 8+2i, 9+2i; O rows (slots) 32q..32q+31 of every group.
+        const int q = warp - kSoftWarp0;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const int r = lane >> 2, i4 = lane & 3;
+        const int rows[2] = {16 * q + r, 16 * q + r + 8};
+        const int heads[4] = {2 * i4, 2 * i4 + 1, 8 + 2 * i4, 9 + 2 * i4};
+        float m_ref[4], l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) { m_ref[e] = -INFINITY; l[e] = 0.f; }
+        long long pid_next = page_id(args, b, page_of(0));
+        for (int i = 0; i < T; ++i) {
+            const int bi = i & 1;
+            const bool vpage = page_ok(args, pid_next);
+            if (i + 1 < T) pid_next = page_id(args, b, page_of(i + 1));
+            mbar_wait(smem_u32(&sm.sfull[bi]), (unsigned)((i >> 1) & 1), &sm.abort);
+            __syncwarp();
+            tc_fence_after();
+            uint32_t u[8];
+            asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+                           "=r"(u[7])
+                         : "r"(tmem + lane_base + kSCol + 16 * bi));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.sfree[bi]));
+            // s[e][j]: head heads[e], row rows[j]
+            float s2[4][2];
+            bool up = false;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const bool valid = vpage && page_of(i) * kPageTok + rows[j] < L;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t raw = u[(e >> 1) * 4 + 2 * j + (e & 1)];
+                    s2[e][j] = valid ? __uint_as_float(raw) * args.scale_log2 : -INFINITY;
+                    up |= s2[e][j] > m_ref[e] + kRescaleLog2 || (m_ref[e] == -INFINITY && s2[e][j] > -INFINITY);
+                }
+            }
+            // the four softmax warps agree on whether any head's reference moves
+            const bool wup = __any_sync(0xffffffffu, up);
+            if (lane == 0) sm.vote[bi][q] = wup ? 1 : 0;
+            named_bar_sync(1, 128);
+            const bool any = (sm.vote[bi][0] | sm.vote[bi][1] | sm.vote[bi][2] | sm.vote[bi][3]) != 0;
+            if (any) {
+                // per-head max over the tile: lanes sharing i4 hold the same heads
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float mx = fmaxf(s2[e][0], s2[e][1]);
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    if (r == 0) sm.red[q][heads[e]] = mx;
+                }
+                named_bar_sync(1, 128);
+                if (q == 0 && lane < 16) {
+                    // one thread per head: new reference and factor for all warps
+                    const int h = lane;
+                    const float tm = fmaxf(fmaxf(sm.red[0][h], sm.red[1][h]), fmaxf(sm.red[2][h], sm.red[3][h]));
+                    const float mo = sm.mref[h];
+                    float al = 1.f, mn = mo;
+                    if (tm > mo + kRescaleLog2 || (mo == -INFINITY && tm > -INFINITY)) {
+                        al = (mo == -INFINITY) ? 0.f : ex2(mo - tm);
+                        mn = tm;
+                    }
+                    sm.alpha[h] = al;
+                    sm.mref[h] = mn;
+                }
+                named_bar_sync(1, 128);
+                bool moved = false;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float al = sm.alpha[heads[e]];
+                    m_ref[e] = sm.mref[heads[e]];
+                    l[e] *= al;
+                }
+#pragma unroll
+                for (int h = 0; h < 16; ++h) moved |= sm.alpha[h] != 1.f;
+                if (moved && i > 0) {
+                    // O holds PV of tiles 0..i-1: wait for PV(i-1), scale this quarter's lanes
+                    mbar_wait(smem_u32(&sm.xfree[(i - 1) & 1]), (unsigned)(((i - 1) >> 1) & 1), &sm.abort);
+                    __syncwarp();
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int g = 0; g < 4; ++g) {
+                        uint32_t v[16];
+                        tmem_ld16(tmem + lane_base + kOCol + 16 * g, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int h = 0; h < 16; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * sm.alpha[h]);
+                        tmem_st16(tmem + lane_base + kOCol + 16 * g, v);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                }
+                named_bar_sync(1, 128);        // red / alpha are read by every softmax warp before reuse
+            }
+            // P buffer bi is free once PV(i - 2) has completed
+            if (i >= 2) mbar_wait(smem_u32(&sm.xfree[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
+            uint8_t* P = sm.P[bi];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float p = (m_ref[e] == -INFINITY) ? 0.f : ex2(s2[e][j] - m_ref[e]);
+                    l[e] += p;
+                    *reinterpret_cast<__half*>(P + plain_off(heads[e], rows[j], 8 * 128)) = __float2half_rn(p);
+                }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.pready[bi]));
+        }
+        // ---- this item's partial: O (rows = slots), per-head (m, l) ----------------
+        if (T > 0) mbar_wait(smem_u32(&sm.xfree[(T - 1) & 1]), (unsigned)(((T - 1) >> 1) & 1), &sm.abort);
+        __syncwarp();
         tc_fence_after();
-    }
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 4);
-    if (jj == 0) sm.team_ml[team][hh] = make_float2(m_ref, l_part);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
-    // ---- merge the teams: warp q of team t writes channel groups t, t + kTeams, ... ----
-    {
-        float Mx[16];
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-            float m = sm.team_ml[0][h].x;
-#pragma unroll
-            for (int t = 1; t < kTeams; ++t) m = fmaxf(m, sm.team_ml[t][h].x);
-            Mx[h] = m;
-        }
-        const int ks = lane >> 4, y = lane & 15;
-        const int chq = 32 * q + 8 * ((y & 7) >> 1) + 4 * (y & 1) + 2 * ks + (y >> 3);
+        const int m = 32 * q + lane;           // O row = slot within the group
 #pragma unroll 1
-        for (int g = team; g < 4; g += kTeams) {
-            float acc[16];
+        for (int g = 0; g < 4; ++g) {
+            uint32_t v[16];
+            tmem_ld16(tmem + lane_base + kOCol + 16 * g, v);
+            tmem_ld_wait();
+            float* dst = args.ws_o + ((size_t)blockIdx.x * args.heads + h0) * ROLAQ_D_C + 128 * g + slot_channel(m);
 #pragma unroll
-            for (int h = 0; h < 16; ++h) acc[h] = 0.f;
-#pragma unroll 1
-            for (int t = 0; t < kTeams; ++t) {
-                float w[16];
-                bool any = false;
-#pragma unroll
-                for (int h = 0; h < 16; ++h) {
-                    const float m = sm.team_ml[t][h].x;
-                    w[h] = (m == -INFINITY) ? 0.f : ex2(m - Mx[h]);
-                    any |= w[h] != 0.f;
-                }
-                if (any) {                           // the same for every lane of the warp
-                    uint32_t u[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * q) << 16) + t * kTeamCols + 16 * g, u);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int h = 0; h < 16; ++h)
-                        if (w[h] != 0.f) acc[h] = fmaf(w[h], __uint_as_float(u[h]), acc[h]);
-                }
-            }
-            float* dst = args.ws_o + ((size_t)blockIdx.x * args.heads + h0) * ROLAQ_D_C + 128 * g + chq;
-#pragma unroll
-            for (int h = 0; h < 16; ++h) dst[(size_t)h * ROLAQ_D_C] = acc[h];
+            for (int h = 0; h < 16; ++h) dst[(size_t)h * ROLAQ_D_C] = __uint_as_float(v[h]);
         }
-        if (team == 0 && q == 0 && lane < 16) {
-            float m = sm.team_ml[0][lane].x;
-            for (int t = 1; t < kTeams; ++t) m = fmaxf(m, sm.team_ml[t][lane].x);
-            float l = 0.f;
-            for (int t = 0; t < kTeams; ++t) {
-                const float2 ml = sm.team_ml[t][lane];
-                if (ml.x != -INFINITY) l += ex2(ml.x - m) * ml.y;
-            }
-            args.ws_ml[(size_t)blockIdx.x * args.heads + h0 + lane] = make_float2(m, l);
+        // row sums: lanes sharing i4 (8 per warp) and the four warps
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float v = l[e];
+            v += __shfl_xor_sync(0xffffffffu, v, 4);
+            v += __shfl_xor_sync(0xffffffffu, v, 8);
+            v += __shfl_xor_sync(0xffffffffu, v, 16);
+            if (r == 0) sm.red[q][heads[e]] = v;
+        }
+        named_bar_sync(1, 128);
+        if (q == 0 && lane < 16) {
+            const int h = lane;
+            args.ws_ml[(size_t)blockIdx.x * args.heads + h0 + h] =
+                make_float2(sm.mref[h], (sm.red[0][h] + sm.red[1][h]) + (sm.red[2][h] + sm.red[3][h]));
         }
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" :: "r"(tmem) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
