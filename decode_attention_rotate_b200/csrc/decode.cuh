@@ -74,8 +74,8 @@ struct DecodeSmem {
     int vote[2][4];
     alignas(8) uint64_t full[kStages];     // page copy landed
     alignas(8) uint64_t pfree[kStages];    // page read by the dequant warps and the QK MMAs
-    alignas(8) uint64_t xready[2];         // x tile written
-    alignas(8) uint64_t xfree[2];          // PV of the tile done (x tile and P buffer free)
+    alignas(8) uint64_t xready[2][2];      // x tile half written (channel groups 0-1 / 2-3)
+    alignas(8) uint64_t xfree[2][2];       // PV of the tile done for groups 0-1 / all groups
     alignas(8) uint64_t sfull[2];          // QK of the tile done
     alignas(8) uint64_t sfree[2];          // scores read by the softmax warps
     alignas(8) uint64_t pready[2];         // P written (and O rescaled if needed)
@@ -334,8 +334,10 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             mbar_init(smem_u32(&sm.pfree[s]), (kDecodeThreads / 32 - kDqWarp0) + 1);
         }
         for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_u32(&sm.xready[s]), kDecodeThreads / 32 - kDqWarp0);
-            mbar_init(smem_u32(&sm.xfree[s]), 1);
+            for (int hf = 0; hf < 2; ++hf) {
+                mbar_init(smem_u32(&sm.xready[s][hf]), (kDecodeThreads / 32 - kDqWarp0) / 2);
+                mbar_init(smem_u32(&sm.xfree[s][hf]), 1);
+            }
             mbar_init(smem_u32(&sm.sfull[s]), 1);
             mbar_init(smem_u32(&sm.sfree[s]), 4);
             mbar_init(smem_u32(&sm.pready[s]), 4);
@@ -413,43 +415,56 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                 const uint32_t first = j > 0 ? 1u : 0u;
                 if (elect_one()) {
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
+                    for (int g = 0; g < 4; ++g) {
 #pragma unroll
                         for (int ks = 0; ks < kPageTok / 16; ++ks)
                             umma_ss1(tmem + kOCol + 16 * g, da + (uint64_t)((2 * g * kXAtom + ks * 2048) >> 4),
                                      db + (uint64_t)((ks * 256) >> 4), kIdPv, ks > 0 ? 1u : first);
-                    umma_commit(smem_u32(&sm.xfree[bj]));
+                        if (g == 1) umma_commit(smem_u32(&sm.xfree[bj][0]));   // groups 0-1 read
+                    }
+                    umma_commit(smem_u32(&sm.xfree[bj][1]));
                 }
                 __syncwarp();
             };
             for (int i = 0; i < T; ++i) {
                 const int bi = i & 1, st = i % kStages;
-                mbar_wait(smem_u32(&sm.xready[bi]), (unsigned)((i >> 1) & 1), &sm.abort);
                 if (i >= 2) mbar_wait(smem_u32(&sm.sfree[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
-                __syncwarp();
-                tc_fence_after();
                 const uint64_t da = dxk + (uint64_t)(bi * (kXTile >> 4));
                 const uint64_t dk = dkr + (uint64_t)(st * (ROLAQ_PAGE_BYTES >> 4));
                 const uint32_t d = tmem + kSCol + 16 * bi;
-                if (elect_one()) {
+                // channel groups 0-1 (K steps 0..15) as soon as that half of the tile is written
 #pragma unroll
-                    for (int kk = 0; kk < ROLAQ_D_C / 16; ++kk)
-                        umma_ss1(d, da + (uint64_t)(((kk >> 2) * kXAtom + (kk & 3) * 32) >> 4),
-                                 dqc + (uint64_t)((kk * 256) >> 4), kIdQk, kk > 0 ? 1u : 0u);
+                for (int hf = 0; hf < 2; ++hf) {
+                    mbar_wait(smem_u32(&sm.xready[bi][hf]), (unsigned)((i >> 1) & 1), &sm.abort);
+                    __syncwarp();
+                    tc_fence_after();
+                    if (elect_one()) {
 #pragma unroll
-                    for (int kk = 0; kk < ROLAQ_D_R / 16; ++kk)
-                        umma_ss1(d, dk + (uint64_t)((kk * 32) >> 4), dqr + (uint64_t)((kk * 256) >> 4), kIdRope, 1u);
-                    umma_commit(smem_u32(&sm.sfull[bi]));
-                    umma_commit(smem_u32(&sm.pfree[st]));
+                        for (int k2 = 0; k2 < ROLAQ_D_C / 32; ++k2) {
+                            const int kk = hf * (ROLAQ_D_C / 32) + k2;
+                            umma_ss1(d, da + (uint64_t)(((kk >> 2) * kXAtom + (kk & 3) * 32) >> 4),
+                                     dqc + (uint64_t)((kk * 256) >> 4), kIdQk, kk > 0 ? 1u : 0u);
+                        }
+                        if (hf == 1) {
+#pragma unroll
+                            for (int kk = 0; kk < ROLAQ_D_R / 16; ++kk)
+                                umma_ss1(d, dk + (uint64_t)((kk * 32) >> 4), dqr + (uint64_t)((kk * 256) >> 4),
+                                         kIdRope, 1u);
+                            umma_commit(smem_u32(&sm.sfull[bi]));
+                            umma_commit(smem_u32(&sm.pfree[st]));
+                        }
+                    }
+                    __syncwarp();
                 }
-                __syncwarp();
                 if (i >= 1) pv(i - 1);
             }
             if (T > 0) pv(T - 1);
         }
     } else if (warp >= kDqWarp0) {
         // ------------------------------------------------------------- dequant ----
-        const int t = 8 * (warp - kDqWarp0) + (lane & 7), g = lane >> 3;
+        // warps 8..11 take channel groups 0-1, warps 12..15 groups 2-3
+        const int wq = warp - kDqWarp0, hf = wq >> 2;
+        const int t = 16 * (wq & 3) + (lane & 15), g = 2 * hf + (lane >> 4);
         const bool protect = args.n_sink > 0 || args.n_recent > 0;
         const int nslot = args.n_sink + args.n_recent;
         const float la = args.level_a, lb = args.level_b;
@@ -468,11 +483,11 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             dequant_tile_part(sm.stage[st], t, g, valid, prot, prow, la, lb, o);
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.pfree[st]));      // this warp is done with the page
-            if (i >= 2) mbar_wait(smem_u32(&sm.xfree[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
+            if (i >= 2) mbar_wait(smem_u32(&sm.xfree[bi][hf]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
             store_tile_part(sm.x[bi], t, g, o);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.xready[bi]));
+            if (lane == 0) mbar_arrive(smem_u32(&sm.xready[bi][hf]));
         }
     } else if (warp >= kSoftWarp0) {
         // ------------------------------------------------------------- softmax ----
@@ -558,7 +573,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                 for (int h = 0; h < 16; ++h) moved |= sm.alpha[h] != 1.f;
                 if (moved && i > 0) {
                     // O holds PV of tiles 0..i-1: wait for PV(i-1), scale this quarter's lanes
-                    mbar_wait(smem_u32(&sm.xfree[(i - 1) & 1]), (unsigned)(((i - 1) >> 1) & 1), &sm.abort);
+                    mbar_wait(smem_u32(&sm.xfree[(i - 1) & 1][1]), (unsigned)(((i - 1) >> 1) & 1), &sm.abort);
                     __syncwarp();
                     tc_fence_after();
 #pragma unroll 1
@@ -576,7 +591,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                 named_bar_sync(1, 128);        // red / alpha are read by every softmax warp before reuse
             }
             // P buffer bi is free once PV(i - 2) has completed
-            if (i >= 2) mbar_wait(smem_u32(&sm.xfree[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
+            if (i >= 2) mbar_wait(smem_u32(&sm.xfree[bi][1]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
             uint8_t* P = sm.P[bi];
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -591,7 +606,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             if (lane == 0) mbar_arrive(smem_u32(&sm.pready[bi]));
         }
         // ---- this item's partial: O (rows = slots), per-head (m, l) ----------------
-        if (T > 0) mbar_wait(smem_u32(&sm.xfree[(T - 1) & 1]), (unsigned)(((T - 1) >> 1) & 1), &sm.abort);
+        if (T > 0) mbar_wait(smem_u32(&sm.xfree[(T - 1) & 1][1]), (unsigned)(((T - 1) >> 1) & 1), &sm.abort);
         __syncwarp();
         tc_fence_after();
         const int m = 32 * q + lane;           // O row = slot within the group
