@@ -288,3 +288,34 @@ def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
 
 def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return (np.ascontiguousarray(bf16_round(x).astype(np.float32)).view(np.uint32) >> 16).astype(np.uint16)
+
+
+# ---- absorbed projections around the cache (RoLaQ §3.3; Fig. 3a) -----------------
+# In absorbed MLA, head h's no-RoPE key and value are k_h = c . W_UK[h] and
+# v_h = c . W_UV[h] (c the 512-d content latent, W_* [512][128]).  A query's no-RoPE score
+# q_h . k_h = (q_h . W_UK[h]^T) . c, and with the cache holding y = c . R (R orthogonal,
+# c = y . R^T) this is (q_h . W_UK[h]^T . R) . y: the read-side rotation folds into the
+# query projection.  The attention output over y, o_rot = sum_t p_t y_t, gives head h's
+# value output sum_t p_t v_t = o_rot . R^T . W_UV[h]: the inverse rotation folds into the
+# value projection.
+
+def fold_weights(W_UK: np.ndarray, W_UV: np.ndarray, R: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """W_UK, W_UV [H][512][128], R [512][512] (y = c . R) -> W_q [H][128][512] = W_UK[h]^T . R
+    and W_o [H][512][128] = R^T . W_UV[h], in fp64."""
+    W_UK = np.asarray(W_UK, np.float64)
+    W_UV = np.asarray(W_UV, np.float64)
+    R = np.asarray(R, np.float64)
+    W_q = np.stack([W_UK[h].T @ R for h in range(W_UK.shape[0])])
+    W_o = np.stack([R.T @ W_UV[h] for h in range(W_UV.shape[0])])
+    return W_q, W_o
+
+
+def fold_query(q_nope: np.ndarray, W_q: np.ndarray) -> np.ndarray:
+    """q_nope [B][H][128] -> q_c_rot [B][H][512] = q_nope[b,h] . W_q[h]."""
+    q_nope = np.asarray(q_nope, np.float64)
+    return np.einsum("bhn,hnj->bhj", q_nope, np.asarray(W_q, np.float64))
+
+
+def unfold_output(out_rot: np.ndarray, W_o: np.ndarray) -> np.ndarray:
+    """out_rot [B][H][512] (rotated basis) -> v [B][H][128] = out_rot[b,h] . W_o[h]."""
+    return np.einsum("bhk,hkn->bhn", np.asarray(out_rot, np.float64), np.asarray(W_o, np.float64))

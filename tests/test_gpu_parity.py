@@ -361,3 +361,40 @@ def test_streaming_append_with_recent_ring():
         o_ref, _ = O.decode_request(f64(q_c[r]), f64(q_r[r]), packed, meta, O.bf16_bits_to_f64(krb), tau,
                                     SM_SCALE, content, n_sink, n_recent)
         assert rel_l2(out[r], o_ref).max() <= DECODE_TOL
+
+
+def test_decode_fp16_range_status():
+    """x and the content query enter the decode MMAs as fp16: a cache whose decoded values
+    pass 65504, or a query element that large, sets ROLAQ_STATUS_RANGE (the result of that
+    call is not valid); an ordinary call leaves the status clean."""
+    w = W.Workload("range", 1, (200,), 16, seed=97)
+    tau, gain = 0.95, 1.1
+    Rm = W.rotation(w.seed)
+    R_split = R.prepare_rotation(torch.as_tensor(Rm).to(DEV))
+    pt = W.page_table(w)
+    p = R.layer_params_init(tau, gain)
+    lens = torch.tensor([200], dtype=torch.int32, device=DEV)
+    q_c, q_r = W.queries(w, 0)
+    q_c, q_r = q_c.to(DEV), q_r.to(DEV)
+    req = torch.zeros(200, dtype=torch.int32, device=DEV)
+    pos = torch.arange(200, dtype=torch.int32, device=DEV)
+    kr = W.rope_key(w, 0, 200).to(DEV)
+
+    def cache_with(scale):
+        cache = R.PagedCache(int(pt.max()) + 1, torch.as_tensor(pt), device=DEV)
+        c = (W.latent(w, 0, 200).float() * scale).to(torch.bfloat16).to(DEV)
+        R.quantize_append(cache, p, R_split, c, kr, req, pos, lens)
+        return cache
+
+    assert R.get_status() == 0
+    ok = cache_with(1.0)
+    R.decode_attn(ok, p, q_c, q_r, lens, SM_SCALE)
+    assert R.get_status() == 0
+    big = cache_with(1.0e5)
+    R.decode_attn(big, p, q_c, q_r, lens, SM_SCALE)
+    assert R.get_status() & R.STATUS_RANGE
+    q_big = q_c.clone()
+    q_big[0, 3, 17] = 1.0e5
+    R.decode_attn(ok, p, q_big, q_r, lens, SM_SCALE)
+    assert R.get_status() & R.STATUS_RANGE
+    assert R.get_status() == 0

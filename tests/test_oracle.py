@@ -400,3 +400,66 @@ def test_planted_transposed_rotation_is_caught(monkeypatch):
     monkeypatch.setattr(O, "rotate", lambda c, R: np.asarray(c, np.float64) @ np.asarray(R, np.float64).T)
     with pytest.raises(AssertionError):
         test_quantization_disabled_reduces_to_standard_mla()
+
+
+# ---- absorbed projections (query fold / output unfold) ----------------------------
+
+def _mla_weights(seed, H=4):
+    rng = np.random.default_rng(seed)
+    W_UK = rng.standard_normal((H, O.D_C, 128)) / math.sqrt(O.D_C)
+    W_UV = rng.standard_normal((H, O.D_C, 128)) / math.sqrt(O.D_C)
+    q, r = np.linalg.qr(rng.standard_normal((O.D_C, O.D_C)))
+    return W_UK, W_UV, q * np.sign(np.diag(r))[None, :]
+
+
+def test_fold_query_preserves_no_rope_scores():
+    """q . (c W_UK)^T must equal fold(q) . (c R)^T for every token: the fold is exactly the
+    read-side rotation absorbed into the query projection."""
+    W_UK, W_UV, R = _mla_weights(3)
+    rng = np.random.default_rng(4)
+    c = rng.standard_normal((50, O.D_C))
+    q = rng.standard_normal((2, 4, 128))
+    W_q, _ = O.fold_weights(W_UK, W_UV, R)
+    qt = O.fold_query(q, W_q)
+    y = O.rotate(c, R)
+    for b in range(2):
+        for h in range(4):
+            direct = q[b, h] @ (c @ W_UK[h]).T
+            folded = qt[b, h] @ y.T
+            assert np.allclose(folded, direct, rtol=1e-12, atol=1e-12)
+
+
+def test_unfold_output_recovers_values():
+    """sum_t p_t (c_t W_UV) must equal unfold(sum_t p_t y_t)."""
+    W_UK, W_UV, R = _mla_weights(5)
+    rng = np.random.default_rng(6)
+    c = rng.standard_normal((40, O.D_C))
+    p = rng.dirichlet(np.ones(40), size=(2, 4))          # [2][4][40] attention weights
+    y = O.rotate(c, R)
+    _, W_o = O.fold_weights(W_UK, W_UV, R)
+    out_rot = np.einsum("bht,tk->bhk", p, y)
+    v = O.unfold_output(out_rot, W_o)
+    for b in range(2):
+        for h in range(4):
+            assert np.allclose(v[b, h], p[b, h] @ (c @ W_UV[h]), rtol=1e-12, atol=1e-12)
+
+
+def test_fold_with_identity_rotation_is_transpose():
+    W_UK, W_UV, _ = _mla_weights(7, H=2)
+    W_q, W_o = O.fold_weights(W_UK, W_UV, np.eye(O.D_C))
+    assert np.array_equal(W_q, np.transpose(W_UK, (0, 2, 1)))
+    assert np.array_equal(W_o, W_UV)
+
+
+def test_planted_fold_mistake_is_caught(monkeypatch):
+    """Folding R^T instead of R into the query breaks the score identity."""
+    W_UK, W_UV, R = _mla_weights(8, H=1)
+    orig = O.fold_weights
+    monkeypatch.setattr(O, "fold_weights", lambda a, b, r: orig(a, b, np.asarray(r).T))
+    rng = np.random.default_rng(9)
+    c = rng.standard_normal((10, O.D_C))
+    q = rng.standard_normal((1, 1, 128))
+    W_q, _ = O.fold_weights(W_UK, W_UV, R)
+    folded = O.fold_query(q, W_q)[0, 0] @ O.rotate(c, R).T
+    direct = q[0, 0] @ (c @ W_UK[0]).T
+    assert not np.allclose(folded, direct, rtol=1e-6, atol=1e-6)
