@@ -277,6 +277,8 @@ def run_ours(args, rank, world, dev):
     # prefill write path: 65,536 tokens x 27 layers
     q_stats = bench_quantize(args, dev, world)
     bf16_stats = bench_bf16_baseline(args, dev, world, w, dec_ms)
+    proj_stats = [bench_projections(args, dev, world, w.batch, w.heads),
+                  bench_projections(args, dev, world, W.PAGED_H128.batch, W.PAGED_H128.heads)]
     clocks = sampler.stop()     # sampled across the timed regions
 
     hbm, bf16, src = peaks()
@@ -302,6 +304,7 @@ def run_ours(args, rank, world, dev):
         "gpu_launches": args.steps * w.layers * 3,
         "quantize": q_stats,
         "bf16_baseline": bf16_stats,
+        "projections": proj_stats,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -356,6 +359,51 @@ def bench_quantize(args, dev, world):
                     "frac": round(bytes_ / (per_launch_ms * 1e-3) / 1e9 / hbm, 4)}}
 
 
+# ------------------------------------------------------ absorbed projections ----
+# Per decode step and layer: the query fold before the cache read and the output unfold
+# after it, over one set of folded bf16 weights per layer; enough layers that the weights
+# of one sweep exceed L2 (every call reads its weights from HBM).
+
+def bench_projections(args, dev, world, batch, heads):
+    per_layer = 2 * heads * R.D_NOPE * R.D_C * 2                   # W_q + W_o, bf16
+    layers = max(27, -(-300_000_000 // per_layer))                 # > 2 x the 126 MB L2
+    g = W.device_generator(4242 + heads, dev)
+    Wq = [(torch.randn((heads, R.D_NOPE, R.D_C), generator=g, device=dev) / 11.3).to(torch.bfloat16)
+          for _ in range(layers)]
+    Wo = [(torch.randn((heads, R.D_C, R.D_V), generator=g, device=dev) / 22.6).to(torch.bfloat16)
+          for _ in range(layers)]
+    q = torch.randn((batch, heads, R.D_NOPE), generator=g, device=dev).to(torch.bfloat16)
+    o = torch.randn((batch, heads, R.D_C), generator=g, device=dev)
+    qc = torch.empty((batch, heads, R.D_C), dtype=torch.bfloat16, device=dev)
+    v = torch.empty((batch, heads, R.D_V), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def sweep():
+        for l in range(layers):
+            R.fold_query(q, Wq[l], out=qc)
+            R.unfold_output(o, Wo[l], v=v)
+
+    for _ in range(max(args.warmup, 3)):
+        sweep()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    reps = 5
+    t0.record(stream)
+    for _ in range(reps):
+        sweep()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    us = t0.elapsed_time(t1) * 1e3 / (reps * layers)               # one fold + one unfold
+    bytes_ = per_layer + batch * heads * (R.D_NOPE * 2 + R.D_C * 2 + R.D_C * 4 + R.D_V * 4)
+    hbm, _, src = peaks()
+    gbs = bytes_ / (us * 1e-6) / 1e9
+    return {"batch": batch, "heads": heads, "us_per_layer": round(us, 3), "bytes_per_layer": bytes_,
+            "layers_swept": layers, "launches_per_layer": 2,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "peak_source": src}}
+
+
 # ------------------------------------------------------------- BF16 baseline ----
 # The same decode on an uncompressed cache (1,152 B per token: 512 bf16 latent + 64 bf16
 # RoPE key, 64-token pages), run by a library kernel: FlashInfer's TRT-LLM-generated MLA
@@ -408,7 +456,8 @@ def bench_bf16_baseline(args, dev, world, w, dec_ms):
 # ------------------------------------------------------------ profiling cases ----
 # Small single-kernel cases for ncu captures (inputs larger than L2, a few hundred MB on
 # the device): `--case decode` runs one layer of 4 requests x 131,072 tokens at 16 heads,
-# `--case quantize` the write path on 262,144 tokens.  They print their own timing.
+# `--case quantize` the write path on 262,144 tokens, `--case project` the query fold and
+# output unfold for 32 requests x 128 heads.  They print their own timing.
 
 def run_case(args, dev):
     if args.case == "decode":
@@ -419,6 +468,27 @@ def run_case(args, dev):
         lens = torch.as_tensor(w.seq_lens, dtype=torch.int32, device=dev)
         fn = lambda: R.decode_attn(lay.cache, lay.params, lay.q_c, lay.q_r, lens, SM_SCALE, lay.out, lay.lse, ws)
         nbytes = w.total_tokens * R.TOKEN_BYTES
+    elif args.case == "project":
+        # query fold + output unfold, 32 requests x 128 heads, ten layers' weights in turn
+        B, H, nl = 32, 128, 10
+        g = W.device_generator(4244, dev)
+        Wq = [(torch.randn((H, R.D_NOPE, R.D_C), generator=g, device=dev) / 11.3).to(torch.bfloat16)
+              for _ in range(nl)]
+        Wo = [(torch.randn((H, R.D_C, R.D_V), generator=g, device=dev) / 22.6).to(torch.bfloat16)
+              for _ in range(nl)]
+        q = torch.randn((B, H, R.D_NOPE), generator=g, device=dev).to(torch.bfloat16)
+        o = torch.randn((B, H, R.D_C), generator=g, device=dev)
+        qc = torch.empty((B, H, R.D_C), dtype=torch.bfloat16, device=dev)
+        v = torch.empty((B, H, R.D_V), dtype=torch.float32, device=dev)
+        it = [0]
+
+        def fn():
+            l = it[0] % nl
+            it[0] += 1
+            R.fold_query(q, Wq[l], out=qc)
+            R.unfold_output(o, Wo[l], v=v)
+        w = W.Workload("project_b32_h128", B, (1,) * B, H, seed=4244)
+        nbytes = 2 * H * R.D_NOPE * R.D_C * 2 + B * H * (R.D_NOPE * 2 + R.D_C * 2 + R.D_C * 4 + R.D_V * 4)
     else:
         w = W.Workload("quantize_262k", 1, (262144,), 16, seed=4243)
         n = w.total_tokens
@@ -509,7 +579,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["decode", "quantize"], default=None,
+    ap.add_argument("--case", choices=["decode", "quantize", "project"], default=None,
                     help="run one small single-kernel case (for ncu captures) instead of the bench")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 1)

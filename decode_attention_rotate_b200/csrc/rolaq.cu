@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "project.cuh"
 #include "quantize.cuh"
 
 using namespace rolaq;
@@ -317,6 +318,44 @@ int rolaq_decode_attn_static(const rolaq_cache* cache, const rolaq_layer_params*
     if (!scratch) return ROLAQ_ECUDA;
     return rolaq_decode_attn(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale,
                              out_dev, lse_dev, scratch, (size_t)ROLAQ_STATIC_SCRATCH_BYTES, stream);
+}
+
+int rolaq_fold_weights(const float* W_UK_dev, const float* W_UV_dev, const float* R_dev,
+                       int heads, void* W_q_dev, void* W_o_dev, void* stream) {
+    if (!W_UK_dev || !W_UV_dev || !R_dev || !W_q_dev || !W_o_dev || heads <= 0 || heads > 65535)
+        return ROLAQ_EINVAL;
+    if (!aligned(W_UK_dev, 4) || !aligned(W_UV_dev, 4) || !aligned(R_dev, 4) || !aligned(W_q_dev, 16) ||
+        !aligned(W_o_dev, 16))
+        return ROLAQ_EINVAL;
+    cudaStream_t s = (cudaStream_t)stream;
+    rolaq_fold_wq<<<dim3(ROLAQ_D_C / kFoldThreads, ROLAQ_D_NOPE, heads), kFoldThreads, 0, s>>>(
+        W_UK_dev, R_dev, static_cast<__nv_bfloat16*>(W_q_dev));
+    rolaq_fold_wo<<<dim3(ROLAQ_D_C, heads), kFoldThreads, 0, s>>>(W_UV_dev, R_dev,
+                                                                   static_cast<__nv_bfloat16*>(W_o_dev));
+    return launch_status();
+}
+
+int rolaq_fold_query(const void* q_nope_dev, const void* W_q_dev, int batch, int heads, void* q_c_rot_dev,
+                     void* stream) {
+    if (heads <= 0 || heads > 65535 || batch < 0) return ROLAQ_EINVAL;
+    if (batch == 0) return ROLAQ_OK;
+    if (!q_nope_dev || !W_q_dev || !q_c_rot_dev) return ROLAQ_EINVAL;
+    if (!aligned(q_nope_dev, 2) || !aligned(W_q_dev, 16) || !aligned(q_c_rot_dev, 2)) return ROLAQ_EINVAL;
+    rolaq_fold_query_kernel<<<dim3(ROLAQ_D_C / kFqCols, heads), kFqThreads, 0, (cudaStream_t)stream>>>(
+        static_cast<const __nv_bfloat16*>(q_nope_dev), static_cast<const __nv_bfloat16*>(W_q_dev), batch, heads,
+        static_cast<__nv_bfloat16*>(q_c_rot_dev));
+    return launch_status();
+}
+
+int rolaq_unfold_output(const float* out_dev, const void* W_o_dev, int batch, int heads, float* v_dev,
+                        void* stream) {
+    if (heads <= 0 || heads > 65535 || batch < 0) return ROLAQ_EINVAL;
+    if (batch == 0) return ROLAQ_OK;
+    if (!out_dev || !W_o_dev || !v_dev) return ROLAQ_EINVAL;
+    if (!aligned(out_dev, 4) || !aligned(W_o_dev, 16) || !aligned(v_dev, 4)) return ROLAQ_EINVAL;
+    rolaq_unfold_output_kernel<<<dim3(kUoSplit, heads), kUoThreads, 0, (cudaStream_t)stream>>>(
+        out_dev, static_cast<const __nv_bfloat16*>(W_o_dev), batch, heads, v_dev);
+    return launch_status();
 }
 
 int rolaq_get_status(int* bits, void* stream) {

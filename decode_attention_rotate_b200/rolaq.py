@@ -18,6 +18,8 @@ from . import build as _build
 
 D_C = 512
 D_R = 64
+D_NOPE = 128            # per-head no-RoPE query width
+D_V = 128               # per-head value width
 PAGE_TOKENS = 64
 PAGE_BYTES = 18432
 TOKEN_BYTES = 288
@@ -91,6 +93,12 @@ def lib() -> ctypes.CDLL:
         L.rolaq_decode_attn_static.restype = i32
         L.rolaq_decode_attn_static.argtypes = [P(rolaq_cache), P(rolaq_layer_params), vp, vp, vp, i32, i32,
                                                ctypes.c_float, vp, vp, vp]
+        L.rolaq_fold_weights.restype = i32
+        L.rolaq_fold_weights.argtypes = [vp, vp, vp, i32, vp, vp, vp]
+        L.rolaq_fold_query.restype = i32
+        L.rolaq_fold_query.argtypes = [vp, vp, i32, i32, vp, vp]
+        L.rolaq_unfold_output.restype = i32
+        L.rolaq_unfold_output.argtypes = [vp, vp, i32, i32, vp, vp]
         L.rolaq_get_status.restype = i32
         L.rolaq_get_status.argtypes = [P(ctypes.c_int), vp]
         _LIB = L
@@ -235,6 +243,47 @@ def decode_attn_static(cache: PagedCache, params: rolaq_layer_params, q_c_rot: t
         ctypes.byref(d), ctypes.byref(params), _ptr(q_c_rot), _ptr(q_r), _ptr(seq_lens), B, H,
         float(sm_scale), _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
+
+
+def fold_weights(W_UK: torch.Tensor, W_UV: torch.Tensor, R: torch.Tensor, stream=None):
+    """rolaq_fold_weights: W_UK, W_UV fp32 [H, 512, 128], R fp32 [512, 512] ->
+    (W_q bf16 [H, 128, 512], W_o bf16 [H, 512, 128])."""
+    H = int(W_UK.shape[0])
+    for t in (W_UK, W_UV, R):
+        assert t.dtype == torch.float32
+    assert tuple(W_UK.shape) == (H, D_C, D_NOPE) and tuple(W_UV.shape) == (H, D_C, D_V)
+    assert tuple(R.shape) == (D_C, D_C)
+    W_q = torch.empty((H, D_NOPE, D_C), dtype=torch.bfloat16, device=W_UK.device)
+    W_o = torch.empty((H, D_C, D_V), dtype=torch.bfloat16, device=W_UK.device)
+    _check("rolaq_fold_weights", lib().rolaq_fold_weights(
+        _ptr(W_UK), _ptr(W_UV), _ptr(R), H, _ptr(W_q), _ptr(W_o), _stream(stream)))
+    return W_q, W_o
+
+
+def fold_query(q_nope: torch.Tensor, W_q: torch.Tensor, out: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """rolaq_fold_query: q_nope bf16 [B, H, 128] -> q_c_rot bf16 [B, H, 512]."""
+    B, H = int(q_nope.shape[0]), int(q_nope.shape[1])
+    assert q_nope.dtype == torch.bfloat16 and tuple(q_nope.shape) == (B, H, D_NOPE)
+    assert W_q.dtype == torch.bfloat16 and tuple(W_q.shape) == (H, D_NOPE, D_C)
+    if out is None:
+        out = torch.empty((B, H, D_C), dtype=torch.bfloat16, device=q_nope.device)
+    _check("rolaq_fold_query", lib().rolaq_fold_query(_ptr(q_nope), _ptr(W_q), B, H, _ptr(out),
+                                                      _stream(stream)))
+    return out
+
+
+def unfold_output(out_rot: torch.Tensor, W_o: torch.Tensor, v: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """rolaq_unfold_output: out_rot fp32 [B, H, 512] -> v fp32 [B, H, 128]."""
+    B, H = int(out_rot.shape[0]), int(out_rot.shape[1])
+    assert out_rot.dtype == torch.float32 and tuple(out_rot.shape) == (B, H, D_C)
+    assert W_o.dtype == torch.bfloat16 and tuple(W_o.shape) == (H, D_C, D_V)
+    if v is None:
+        v = torch.empty((B, H, D_V), dtype=torch.float32, device=out_rot.device)
+    _check("rolaq_unfold_output", lib().rolaq_unfold_output(_ptr(out_rot), _ptr(W_o), B, H, _ptr(v),
+                                                            _stream(stream)))
+    return v
 
 
 def get_status(stream=None) -> int:

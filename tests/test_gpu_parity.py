@@ -237,8 +237,8 @@ def test_decode_single_token_equals_its_reconstruction():
 
 
 def test_end_to_end_write_then_decode():
-    """Cache written by the GPU write path, decoded on the GPU, against the oracle decoding
-    the GPU-written records."""
+    """Cache written by the GPU write path and decoded on the GPU, against the oracle
+    quantizing the same latents itself and decoding its own records."""
     w = W.Workload("e2e", 2, (700, 1333), 16, paged_shuffled=True, seed=95)
     tau, gain = 0.91, 1.13
     lens_l = [700, 1333]
@@ -247,19 +247,11 @@ def test_end_to_end_write_then_decode():
     p = R.layer_params_init(tau, gain)
     lens = torch.as_tensor(lens_l, dtype=torch.int32).to(DEV)
     out, lse = R.decode_attn(cache, p, q_c.to(DEV), q_r.to(DEV), lens, SM_SCALE)
-    pool = cache.pages.cpu().numpy()
-    prot = cache.prot.float().cpu().numpy().astype(np.float64)
-    for r, L in enumerate(lens_l):
-        packed, meta, kr = O.pages_read_fast(pool, pt, r, L)
-        content = np.zeros((L, 512))
-        for pp in range(L):
-            if pp < 4:
-                content[pp] = prot[r, pp]
-            elif pp >= L - 128:
-                content[pp] = prot[r, 4 + pp % 128]
-        o, l = O.decode_request(f64(q_c[r]), f64(q_r[r]), packed, meta, O.bf16_bits_to_f64(kr), tau,
-                                SM_SCALE, content, 4, 128)
-        e = rel_l2(out[r].cpu().numpy().astype(np.float64), o)
+    torch.cuda.synchronize()
+    _, data, _ = build_oracle_cache(w, 0, lens_l, tau, gain, n_sink=4, n_recent=128)
+    o_ref, _ = oracle_decode(data, f64(q_c), f64(q_r), lens_l, tau, SM_SCALE, 4, 128)
+    for r in range(len(lens_l)):
+        e = rel_l2(out[r].cpu().numpy().astype(np.float64), o_ref[r])
         assert e.max() <= DECODE_TOL, e.max()
 
 

@@ -96,3 +96,20 @@ def test_workspace_bytes_shape_rules(lib):
     assert lib.rolaq_decode_workspace_bytes(0, 16) == 0
     n16 = lib.rolaq_decode_workspace_bytes(4, 16)
     assert n16 > 0 and n16 % 16 == 0
+
+
+def test_projection_argument_errors(lib):
+    """Bad pointers and sizes are rejected before any launch; batch == 0 is a no-op."""
+    ptr = 1 << 22
+    fw = lambda a=ptr, b=ptr, r=ptr, h=16, q=ptr, o=ptr: lib.rolaq_fold_weights(a, b, r, h, q, o, None)
+    assert fw(a=None) == -1 and fw(r=None) == -1 and fw(o=None) == -1
+    assert fw(h=0) == -1 and fw(h=-3) == -1
+    assert fw(b=ptr + 2) == -1                                 # fp32 operand not 4-byte aligned
+    fq = lambda q=ptr, w=ptr, b=2, h=16, o=ptr: lib.rolaq_fold_query(q, w, b, h, o, None)
+    assert fq(q=None) == -1 and fq(o=None) == -1 and fq(b=-1) == -1 and fq(h=0) == -1
+    assert fq(q=ptr + 1) == -1                                 # bf16 operand not 2-byte aligned
+    assert fq(b=0) == 0 and fq(b=0, q=None, o=None) == 0
+    uo = lambda o=ptr, w=ptr, b=2, h=16, v=ptr: lib.rolaq_unfold_output(o, w, b, h, v, None)
+    assert uo(o=None) == -1 and uo(v=None) == -1 and uo(b=-1) == -1 and uo(h=0) == -1
+    assert uo(w=ptr + 2) == -1
+    assert uo(b=0) == 0 and uo(b=0, o=None, v=None) == 0
