@@ -173,43 +173,10 @@ __device__ __forceinline__ void dequant_word2(uint32_t w, uint2 la, uint2 lb, ui
 }
 
 // ---- tensor-core operands -----------------------------------------------------
-// Shared-memory matrix descriptor (sm_100 form): start, leading / stride byte offsets
-// (16-byte units), version 1, layout type (0: no swizzle, 2: 128-byte swizzle).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
-}
 // Instruction descriptors: fp32 accumulate, K-major unless noted, N = 16 heads.
 constexpr uint32_t kIdQk = (1u << 4) | ((16u >> 3) << 17) | ((64u >> 4) << 24);                 // f16, M = 64
 constexpr uint32_t kIdRope = kIdQk | (1u << 7) | (1u << 10);                                     // bf16, M = 64
 constexpr uint32_t kIdPv = (1u << 4) | (1u << 15) | ((16u >> 3) << 17) | ((128u >> 4) << 24);   // f16, M = 128, A MN-major
-
-// D (tensor memory) (+)= A (shared memory) * B (shared memory).  Called by a whole warp
-// with warp-uniform operands (so they live in uniform registers); one elected lane issues.
-__device__ __forceinline__ void umma_ss(uint32_t d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
-    asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                 "elect.sync _|e, 0xffffffff;\n\t"
-                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                 :: "r"(d), "l"(da), "l"(db), "r"(idesc), "r"(acc) : "memory");
-}
-// One lane of a converged warp (elect.sync).
-__device__ __forceinline__ bool elect_one() {
-    uint32_t p;
-    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\tselp.u32 %0, 1, 0, e;\n\t}" : "=r"(p));
-    return p != 0;
-}
-// Single-thread forms, for a batch issued inside one elected branch.
-__device__ __forceinline__ void umma_ss1(uint32_t d, uint64_t da, uint64_t db, uint32_t idesc, uint32_t acc) {
-    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-                 :: "r"(d), "l"(da), "l"(db), "r"(idesc), "r"(acc) : "memory");
-}
-// tcgen05.commit from one elected lane of a converged warp.
-__device__ __forceinline__ void umma_commit_warp(uint32_t bar) {
-    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
-                 :: "r"(bar) : "memory");
-}
 
 // Column slot of channel order inside every 16-channel block: the PRMT lookup yields the
 // pairs (k, k+4), so slot 2k + e of a block of 8 holds channel k + 4e.  The query is laid

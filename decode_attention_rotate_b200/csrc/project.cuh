@@ -4,12 +4,8 @@
 //   W_o[h] = R^T . W_UV[h]     [512][128]   (once per layer)
 //   q_c_rot[b,h] = q_nope[b,h] . W_q[h]     (per decode step, bf16 out)
 //   v[b,h]       = out_rot[b,h] . W_o[h]    (per decode step, fp32 out)
-// The folded weights are stored in bf16 (the precision the model's own projections carry)
-// and every sum runs in fp32.  The per-step products are small and bound by reading the
-// weights once: a decode step has a handful of queries per head, so each CTA splits the
-// contraction over its warps (many independent 4- or 8-byte loads in flight per lane),
-// keeps the weights in registers across the batch and reduces the warps' partial sums
-// through shared memory in a fixed order.
+// The folded weights are stored in bf16 (the precision the model's own projections carry);
+// every sum runs in fp32.
 #pragma once
 #include "common.cuh"
 
@@ -41,145 +37,248 @@ rolaq_fold_wo(const float* __restrict__ W_UV, const float* __restrict__ R, __nv_
     W_o[((size_t)h * ROLAQ_D_C + k) * ROLAQ_D_V + n] = __float2bfloat16_rn(acc);
 }
 
-// ---- per step: query fold ---------------------------------------------------------
-// CTA = (64 output columns, head); 8 warps, warp w sums rows n = 16w .. 16w + 15 of W_q,
-// lane l owns columns 2l, 2l + 1 of the CTA's 64 (one 4-byte load per row).
+// ---- per step: query fold and output unfold on the tensor cores ---------------------
+// Both are D[m][b] = sum_k A[m][k] B[b][k] for one head:
+//   fold:   m = 128 output columns j of a 128-column tile, k = n (K = 128), A = W_q[h]^T,
+//           B = q_nope[., h]
+//   unfold: m = the 128 value columns n, k = latent channel (K = 512), A = W_o[h]^T,
+//           B = out[., h] rounded to bf16
+// A is the folded weight read MN-major straight from its row-major layout: a bulk tensor
+// copy of {64 columns x 128 rows} with 128-byte swizzle per block.  B holds up to kPjN
+// queries, K-major in the no-swizzle core-matrix layout (8 rows x 16 bytes per core
+// matrix), written by the CTA's threads; rows past the batch are zero.  One elected lane
+// issues tcgen05.mma (M = 128, N = the queries rounded up to 16, fp32 accumulate in tensor
+// memory) and each of the four warps reads its 32 tensor-memory lanes (32 output rows)
+// in the epilogue.  The weights cross HBM once per call; the MMAs take well under a
+// microsecond, so the kernels run at the weights' read time.
 
-constexpr int kFqThreads = 256;
-constexpr int kFqWarps = kFqThreads / 32;
-constexpr int kFqCols = 64;
-constexpr int kFqRows = ROLAQ_D_NOPE / kFqWarps;    // 16
-constexpr int kFqBatch = 8;                         // queries per pass
+constexpr int kPjThreads = 128;
+constexpr int kPjN = 64;                            // queries per MMA chunk (tensor-memory columns)
+constexpr int kPjBlock = 128 * 128;                 // one {64 columns x 128 rows} bf16 block (16 KB)
+constexpr int kPjStage = 8;                         // 16-byte chunks a thread loads before storing
+// bf16 A and B, fp32 D, A MN-major, M = 128; N is or-ed in per chunk
+constexpr uint32_t kIdProj = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((128u >> 4) << 24);
 
-__global__ void __launch_bounds__(kFqThreads)
-rolaq_fold_query_kernel(const __nv_bfloat16* __restrict__ q_nope, const __nv_bfloat16* __restrict__ W_q,
-                        int batch, int heads, __nv_bfloat16* __restrict__ q_c_rot) {
-    __shared__ float s_q[kFqBatch][ROLAQ_D_NOPE];
-    __shared__ float2 s_part[kFqWarps][kFqBatch][kFqCols / 2];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, h = blockIdx.y;
-    const int col0 = blockIdx.x * kFqCols;
-    const int n0 = warp * kFqRows;
-    float2 w[kFqRows];
-    const __nv_bfloat162* wq = reinterpret_cast<const __nv_bfloat162*>(
-        W_q + ((size_t)h * ROLAQ_D_NOPE + n0) * ROLAQ_D_C + col0) + lane;
+__device__ __forceinline__ uint32_t proj_idesc(int npad) { return kIdProj | ((uint32_t)(npad >> 3) << 17); }
+
+struct FoldQSmem {
+    alignas(1024) uint8_t a[2][kPjBlock];               // W_q tile: columns j0..j0+63, j0+64..j0+127
+    alignas(128) uint8_t b[kPjN / 8][ROLAQ_D_NOPE / 8][128];   // queries: core matrices
+    alignas(8) uint64_t full;
+    alignas(8) uint64_t mma;
+    uint32_t tmem;
+    int abort;
+};
+
+struct UnfoldSmem {
+    alignas(1024) uint8_t a[ROLAQ_D_C / 128][2][kPjBlock];     // W_o: 4 row chunks x 2 column blocks
+    alignas(128) uint8_t b[kPjN / 8][ROLAQ_D_C / 8][128];     // outputs as bf16: core matrices
+    alignas(8) uint64_t full[ROLAQ_D_C / 128];
+    alignas(8) uint64_t mma;
+    uint32_t tmem;
+    int abort;
+};
+
+__device__ __forceinline__ void proj_tmem_alloc(uint32_t* slot) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(slot)), "r"(kPjN) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void proj_tmem_free(uint32_t tmem) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kPjN) : "memory");
+}
+
+// Epilogue: thread (warp w, lane l) owns output row m = 32w + l; columns are queries.
+template <typename Store>
+__device__ __forceinline__ void proj_epilogue(uint32_t tmem, int warp, int npad, Store store) {
+    for (int c0 = 0; c0 < npad; c0 += 16) {
+        uint32_t u[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)c0, u);
+        tmem_ld_wait();
 #pragma unroll
-    for (int i = 0; i < kFqRows; ++i) w[i] = __bfloat1622float2(wq[(size_t)i * (ROLAQ_D_C / 2)]);
-    for (int b0 = 0; b0 < batch; b0 += kFqBatch) {
-        const int nb = min(kFqBatch, batch - b0);
-        for (int e = threadIdx.x; e < kFqBatch * ROLAQ_D_NOPE; e += kFqThreads) {
-            const int bb = e / ROLAQ_D_NOPE, n = e % ROLAQ_D_NOPE;
-            s_q[bb][n] = bb < nb ? __bfloat162float(q_nope[((size_t)(b0 + bb) * heads + h) * ROLAQ_D_NOPE + n]) : 0.f;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int bb = 0; bb < kFqBatch; ++bb) {
-            float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < kFqRows; ++i) {
-                const float q = s_q[bb][n0 + i];
-                acc.x = fmaf(q, w[i].x, acc.x);
-                acc.y = fmaf(q, w[i].y, acc.y);
-            }
-            s_part[warp][bb][lane] = acc;
-        }
-        __syncthreads();
-        // 8 queries x 64 columns = 512 sums of 8 partials, two per thread
-        for (int e = threadIdx.x; e < kFqBatch * kFqCols; e += kFqThreads) {
-            const int bb = e / kFqCols, c = e % kFqCols;
-            if (bb < nb) {
-                float s = 0.f;
-#pragma unroll
-                for (int p = 0; p < kFqWarps; ++p) {
-                    const float2 v = s_part[p][bb][c >> 1];
-                    s += (c & 1) ? v.y : v.x;
-                }
-                q_c_rot[((size_t)(b0 + bb) * heads + h) * ROLAQ_D_C + col0 + c] = __float2bfloat16_rn(s);
-            }
-        }
-        __syncthreads();
+        for (int i = 0; i < 16; ++i) store(c0 + i, __uint_as_float(u[i]));
     }
 }
 
-// ---- per step: output unfold ------------------------------------------------------
-// A cluster of 4 CTAs per head splits K = 512 into quarters.  In each CTA, warp w sums
-// rows 16w .. 16w + 15 of its quarter, lane l owns columns 4l .. 4l + 3 (one 8-byte load
-// per row).  The CTA reduces its warps in shared memory and stores the quarter's sums into
-// the first CTA of the cluster (distributed shared memory), which adds the four quarters
-// in rank order and writes v.
+// grid (512 / 128 column tiles, heads), kPjThreads threads.
+__global__ void __launch_bounds__(kPjThreads)
+rolaq_fold_query_kernel(const __grid_constant__ CUtensorMap map_wq, const __nv_bfloat16* __restrict__ q_nope,
+                        int batch, int heads, __nv_bfloat16* __restrict__ q_c_rot) {
+    extern __shared__ uint8_t smem_raw[];
+    FoldQSmem& sm = *reinterpret_cast<FoldQSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int jt = blockIdx.x, h = blockIdx.y;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&sm.full), 1);
+        mbar_init(smem_u32(&sm.mma), 1);
+        sm.abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&map_wq);
+    }
+    if (warp == 0) proj_tmem_alloc(&sm.tmem);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem;
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(smem_u32(&sm.full), 2 * kPjBlock);
+        for (int c = 0; c < 2; ++c)
+            tma_load_2d(smem_u32(sm.a[c]), &map_wq, jt * 128 + 64 * c, h * ROLAQ_D_NOPE, smem_u32(&sm.full));
+    }
+    const int m = 32 * warp + lane;
+    for (int b0 = 0, it = 0; b0 < batch; b0 += kPjN, ++it) {
+        const int nb = min(kPjN, batch - b0);
+        const int npad = (nb + 15) & ~15;
+        // npad x 16 chunks of 16 bytes: a multiple of the thread count; all of a thread's
+        // loads are issued before its first store
+        constexpr int kCpr = ROLAQ_D_NOPE / 8;
+        for (int e0 = threadIdx.x; e0 < npad * kCpr; e0 += kPjStage * kPjThreads) {
+            uint4 val[kPjStage];
+#pragma unroll
+            for (int u = 0; u < kPjStage; ++u) {
+                const int e = e0 + u * kPjThreads, b = e / kCpr, c = e % kCpr;
+                val[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (b < nb)
+                    val[u] = *reinterpret_cast<const uint4*>(q_nope + ((size_t)(b0 + b) * heads + h) * ROLAQ_D_NOPE + 8 * c);
+            }
+#pragma unroll
+            for (int u = 0; u < kPjStage; ++u) {
+                const int e = e0 + u * kPjThreads, b = e / kCpr, c = e % kCpr;
+                if (b < npad) *reinterpret_cast<uint4*>(&sm.b[b >> 3][c][(b & 7) * 16]) = val[u];
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (warp == 0) {
+            const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.full), 0, &sm.abort));
+            if (ok) {
+                tc_fence_after();
+                const uint32_t idesc = proj_idesc(npad);
+                const uint64_t da = smem_desc(smem_u32(sm.a[0]), kPjBlock, 1024, 2);
+                const uint64_t db = smem_desc(smem_u32(&sm.b[0][0][0]), 128, (ROLAQ_D_NOPE / 8) * 128, 0);
+                if (elect_one()) {
+#pragma unroll
+                    for (int ks = 0; ks < ROLAQ_D_NOPE / 16; ++ks)
+                        umma_ss1(tmem, da + (uint64_t)((ks * 2048) >> 4), db + (uint64_t)((ks * 256) >> 4), idesc,
+                                 ks > 0 ? 1u : 0u);
+                    umma_commit(smem_u32(&sm.mma));
+                }
+                __syncwarp();
+            }
+        }
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.mma), (unsigned)(it & 1), &sm.abort));
+        tc_fence_after();
+        if (ok) {
+            __nv_bfloat16* dst = q_c_rot + (size_t)h * ROLAQ_D_C + jt * 128 + m;
+            proj_epilogue(tmem, warp, npad, [&](int b, float x) {
+                if (b < nb) dst[(size_t)(b0 + b) * heads * ROLAQ_D_C] = __float2bfloat16_rn(x);
+            });
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (sm.abort) break;
+    }
+    tc_fence_after();
+    if (warp == 0) proj_tmem_free(tmem);
+}
 
-constexpr int kUoSplit = 4;                         // CTAs per head (cluster size)
-constexpr int kUoThreads = 256;
-constexpr int kUoWarps = kUoThreads / 32;
-constexpr int kUoK = ROLAQ_D_C / kUoSplit;          // 128 rows of W_o per CTA
-constexpr int kUoRows = kUoK / kUoWarps;            // 16 rows per warp
-constexpr int kUoBatch = 4;                         // outputs per pass
-
-__global__ void __cluster_dims__(kUoSplit, 1, 1) __launch_bounds__(kUoThreads)
-rolaq_unfold_output_kernel(const float* __restrict__ out, const __nv_bfloat16* __restrict__ W_o, int batch,
+// grid (heads), kPjThreads threads.
+__global__ void __launch_bounds__(kPjThreads)
+rolaq_unfold_output_kernel(const __grid_constant__ CUtensorMap map_wo, const float* __restrict__ out, int batch,
                            int heads, float* __restrict__ v) {
-    __shared__ float s_o[kUoBatch][kUoK];
-    __shared__ float4 s_part[kUoWarps][kUoBatch][ROLAQ_D_V / 4];
-    __shared__ float s_red[kUoSplit][kUoBatch][ROLAQ_D_V];   // used in the first CTA
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, h = blockIdx.y;
-    const uint32_t rank = cluster_ctarank();
-    const int kq = (int)rank * kUoK;                 // this CTA's quarter of K
-    const int k0 = warp * kUoRows;                   // this warp's rows inside the quarter
-    uint2 w[kUoRows];                                // packed bf16, widened at use
-    const uint2* wo = reinterpret_cast<const uint2*>(W_o + ((size_t)h * ROLAQ_D_C + kq + k0) * ROLAQ_D_V) + lane;
-#pragma unroll
-    for (int i = 0; i < kUoRows; ++i) w[i] = wo[(size_t)i * (ROLAQ_D_V / 4)];
-    const uint32_t red0 = mapa_shared(smem_u32(&s_red[rank][0][0]), 0);
-    cluster_sync();                                  // every CTA of the cluster is running
-    for (int b0 = 0; b0 < batch; b0 += kUoBatch) {
-        const int nb = min(kUoBatch, batch - b0);
-        for (int e = threadIdx.x; e < kUoBatch * kUoK; e += kUoThreads) {
-            const int bb = e / kUoK, k = e % kUoK;
-            s_o[bb][k] = bb < nb ? out[((size_t)(b0 + bb) * heads + h) * ROLAQ_D_C + kq + k] : 0.f;
+    extern __shared__ uint8_t smem_raw[];
+    UnfoldSmem& sm = *reinterpret_cast<UnfoldSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    constexpr int kChunks = ROLAQ_D_C / 128;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.x;
+    if (threadIdx.x == 0) {
+        for (int c = 0; c < kChunks; ++c) mbar_init(smem_u32(&sm.full[c]), 1);
+        mbar_init(smem_u32(&sm.mma), 1);
+        sm.abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&map_wo);
+    }
+    if (warp == 0) proj_tmem_alloc(&sm.tmem);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem;
+    if (threadIdx.x == 0) {
+        for (int kc = 0; kc < kChunks; ++kc) {
+            mbar_arrive_expect_tx(smem_u32(&sm.full[kc]), 2 * kPjBlock);
+            for (int c = 0; c < 2; ++c)
+                tma_load_2d(smem_u32(sm.a[kc][c]), &map_wo, 64 * c, h * ROLAQ_D_C + 128 * kc, smem_u32(&sm.full[kc]));
         }
-        __syncthreads();
-        float4 acc[kUoBatch];
+    }
+    const int m = 32 * warp + lane;
+    for (int b0 = 0, it = 0; b0 < batch; b0 += kPjN, ++it) {
+        const int nb = min(kPjN, batch - b0);
+        const int npad = (nb + 15) & ~15;
+        // npad x 64 chunks of 8 channels; all of a thread's loads are issued before its
+        // first store
+        constexpr int kCpr = ROLAQ_D_C / 8;
+        for (int e0 = threadIdx.x; e0 < npad * kCpr; e0 += (kPjStage / 2) * kPjThreads) {
+            float4 x0[kPjStage / 2], x1[kPjStage / 2];
 #pragma unroll
-        for (int bb = 0; bb < kUoBatch; ++bb) acc[bb] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int i = 0; i < kUoRows; ++i) {          // widen one row, use it for every output
-            const float w0 = bf16_lo(w[i].x), w1 = bf16_hi(w[i].x), w2 = bf16_lo(w[i].y), w3 = bf16_hi(w[i].y);
-#pragma unroll
-            for (int bb = 0; bb < kUoBatch; ++bb) {
-                const float o = s_o[bb][k0 + i];
-                acc[bb].x = fmaf(o, w0, acc[bb].x);
-                acc[bb].y = fmaf(o, w1, acc[bb].y);
-                acc[bb].z = fmaf(o, w2, acc[bb].z);
-                acc[bb].w = fmaf(o, w3, acc[bb].w);
-            }
-        }
-#pragma unroll
-        for (int bb = 0; bb < kUoBatch; ++bb) s_part[warp][bb][lane] = acc[bb];
-        __syncthreads();
-        // the quarter's 4 x 128 sums (8 warp partials each), two per thread, into the first CTA
-        for (int e = threadIdx.x; e < kUoBatch * ROLAQ_D_V; e += kUoThreads) {
-            const int bb = e / ROLAQ_D_V, c = e % ROLAQ_D_V;
-            float s = 0.f;
-#pragma unroll
-            for (int p = 0; p < kUoWarps; ++p) {
-                const float4 u = s_part[p][bb][c >> 2];
-                s += (c & 3) == 0 ? u.x : (c & 3) == 1 ? u.y : (c & 3) == 2 ? u.z : u.w;
-            }
-            st_cluster_f32(red0 + (uint32_t)e * 4u, s);
-        }
-        cluster_sync();                              // all quarters have landed
-        if (rank == 0) {
-            for (int e = threadIdx.x; e < kUoBatch * ROLAQ_D_V; e += kUoThreads) {
-                const int bb = e / ROLAQ_D_V, c = e % ROLAQ_D_V;
-                if (bb < nb) {
-                    float s = s_red[0][bb][c];
-#pragma unroll
-                    for (int r = 1; r < kUoSplit; ++r) s += s_red[r][bb][c];
-                    v[((size_t)(b0 + bb) * heads + h) * ROLAQ_D_V + c] = s;
+            for (int u = 0; u < kPjStage / 2; ++u) {
+                const int e = e0 + u * kPjThreads, b = e / kCpr, c = e % kCpr;
+                x0[u] = x1[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (b < nb) {
+                    const float4* src = reinterpret_cast<const float4*>(out + ((size_t)(b0 + b) * heads + h) * ROLAQ_D_C + 8 * c);
+                    x0[u] = src[0];
+                    x1[u] = src[1];
                 }
             }
+#pragma unroll
+            for (int u = 0; u < kPjStage / 2; ++u) {
+                const int e = e0 + u * kPjThreads, b = e / kCpr, c = e % kCpr;
+                if (b < npad)
+                    *reinterpret_cast<uint4*>(&sm.b[b >> 3][c][(b & 7) * 16]) =
+                        make_uint4(pack_bf16(x0[u].x, x0[u].y), pack_bf16(x0[u].z, x0[u].w),
+                                   pack_bf16(x1[u].x, x1[u].y), pack_bf16(x1[u].z, x1[u].w));
+            }
         }
-        cluster_sync();                              // the first CTA has read them (next pass reuses)
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (warp == 0) {
+            const uint32_t idesc = proj_idesc(npad);
+            const uint64_t da = smem_desc(smem_u32(sm.a[0][0]), kPjBlock, 1024, 2);
+            const uint64_t db = smem_desc(smem_u32(&sm.b[0][0][0]), 128, (ROLAQ_D_C / 8) * 128, 0);
+            bool ok = true;
+            for (int kc = 0; kc < kChunks && ok; ++kc) {
+                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.full[kc]), 0, &sm.abort));
+                if (ok) {
+                    tc_fence_after();
+                    if (elect_one()) {
+#pragma unroll
+                        for (int s = 0; s < 8; ++s) {
+                            const int ks = 8 * kc + s;
+                            umma_ss1(tmem, da + (uint64_t)((kc * 2 * kPjBlock + s * 2048) >> 4),
+                                     db + (uint64_t)((ks * 256) >> 4), idesc, ks > 0 ? 1u : 0u);
+                        }
+                    }
+                    __syncwarp();
+                }
+            }
+            if (ok) {
+                if (elect_one()) umma_commit(smem_u32(&sm.mma));
+                __syncwarp();
+            }
+        }
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.mma), (unsigned)(it & 1), &sm.abort));
+        tc_fence_after();
+        if (ok) {
+            float* dst = v + (size_t)h * ROLAQ_D_V + m;
+            proj_epilogue(tmem, warp, npad, [&](int b, float x) {
+                if (b < nb) dst[(size_t)(b0 + b) * heads * ROLAQ_D_V] = x;
+            });
+        }
+        tc_fence_before();
+        __syncthreads();
+        if (sm.abort) break;
     }
+    tc_fence_after();
+    if (warp == 0) proj_tmem_free(tmem);
 }
 
 }  // namespace rolaq

@@ -99,6 +99,17 @@ size_t decode_ws_bytes(int batch, int heads) {
     return o + ml;
 }
 
+// Raise a kernel's dynamic shared-memory limit once per device.
+template <typename Kernel>
+void set_smem_limit_once(Kernel k, size_t smem, bool* done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
+    if (!done[dev]) {
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        done[dev] = true;
+    }
+}
+
 int launch_status() {
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? ROLAQ_OK : ROLAQ_ECUDA;
@@ -206,10 +217,8 @@ int rolaq_quantize_append(const rolaq_cache* cache, const rolaq_layer_params* p,
     a.gain = p->gain;
 
     const size_t smem = sizeof(QuantSmem) + 1024;
-    static std::once_flag attr_once;
-    std::call_once(attr_once, [smem] {
-        cudaFuncSetAttribute(rolaq_quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    });
+    static bool attr_done[kMaxDevices] = {false};
+    set_smem_limit_once(rolaq_quantize_kernel, smem, attr_done);
     const int tiles = (n + kQTileM - 1) / kQTileM;
     const int grid = tiles < current_sms() ? tiles : current_sms();
     rolaq_quantize_kernel<<<grid, kQThreads, smem, (cudaStream_t)stream>>>(map_c, map_r, a);
@@ -268,10 +277,8 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
                                         (size_t)items_cap * heads * ROLAQ_D_C * sizeof(float));
 
     const size_t smem = sizeof(DecodeSmem) + 1024;
-    static std::once_flag attr_once;
-    std::call_once(attr_once, [smem] {
-        cudaFuncSetAttribute(rolaq_decode_split, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    });
+    static bool attr_done[kMaxDevices] = {false};
+    set_smem_limit_once(rolaq_decode_split, smem, attr_done);
     cudaStream_t s = (cudaStream_t)stream;
     rolaq_decode_split<<<dim3(items_cap, heads / 16), kDecodeThreads, smem, s>>>(map_page, a);
     if ((rc = launch_status())) return rc;
@@ -340,10 +347,16 @@ int rolaq_fold_query(const void* q_nope_dev, const void* W_q_dev, int batch, int
     if (heads <= 0 || heads > 65535 || batch < 0) return ROLAQ_EINVAL;
     if (batch == 0) return ROLAQ_OK;
     if (!q_nope_dev || !W_q_dev || !q_c_rot_dev) return ROLAQ_EINVAL;
-    if (!aligned(q_nope_dev, 2) || !aligned(W_q_dev, 16) || !aligned(q_c_rot_dev, 2)) return ROLAQ_EINVAL;
-    rolaq_fold_query_kernel<<<dim3(ROLAQ_D_C / kFqCols, heads), kFqThreads, 0, (cudaStream_t)stream>>>(
-        static_cast<const __nv_bfloat16*>(q_nope_dev), static_cast<const __nv_bfloat16*>(W_q_dev), batch, heads,
-        static_cast<__nv_bfloat16*>(q_c_rot_dev));
+    if (!aligned(q_nope_dev, 16) || !aligned(W_q_dev, 16) || !aligned(q_c_rot_dev, 2)) return ROLAQ_EINVAL;
+    CUtensorMap map;
+    if (!encode_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(W_q_dev), ROLAQ_D_C,
+                   (uint64_t)heads * ROLAQ_D_NOPE, ROLAQ_D_C * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return ROLAQ_ECUDA;
+    const size_t smem = sizeof(FoldQSmem) + 1024;
+    static bool attr_done[kMaxDevices] = {false};
+    set_smem_limit_once(rolaq_fold_query_kernel, smem, attr_done);
+    rolaq_fold_query_kernel<<<dim3(ROLAQ_D_C / 128, heads), kPjThreads, smem, (cudaStream_t)stream>>>(
+        map, static_cast<const __nv_bfloat16*>(q_nope_dev), batch, heads, static_cast<__nv_bfloat16*>(q_c_rot_dev));
     return launch_status();
 }
 
@@ -352,9 +365,15 @@ int rolaq_unfold_output(const float* out_dev, const void* W_o_dev, int batch, in
     if (heads <= 0 || heads > 65535 || batch < 0) return ROLAQ_EINVAL;
     if (batch == 0) return ROLAQ_OK;
     if (!out_dev || !W_o_dev || !v_dev) return ROLAQ_EINVAL;
-    if (!aligned(out_dev, 4) || !aligned(W_o_dev, 16) || !aligned(v_dev, 4)) return ROLAQ_EINVAL;
-    rolaq_unfold_output_kernel<<<dim3(kUoSplit, heads), kUoThreads, 0, (cudaStream_t)stream>>>(
-        out_dev, static_cast<const __nv_bfloat16*>(W_o_dev), batch, heads, v_dev);
+    if (!aligned(out_dev, 16) || !aligned(W_o_dev, 16) || !aligned(v_dev, 4)) return ROLAQ_EINVAL;
+    CUtensorMap map;
+    if (!encode_2d(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(W_o_dev), ROLAQ_D_V,
+                   (uint64_t)heads * ROLAQ_D_C, ROLAQ_D_V * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return ROLAQ_ECUDA;
+    const size_t smem = sizeof(UnfoldSmem) + 1024;
+    static bool attr_done[kMaxDevices] = {false};
+    set_smem_limit_once(rolaq_unfold_output_kernel, smem, attr_done);
+    rolaq_unfold_output_kernel<<<heads, kPjThreads, smem, (cudaStream_t)stream>>>(map, out_dev, batch, heads, v_dev);
     return launch_status();
 }
 

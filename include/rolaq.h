@@ -204,14 +204,14 @@ int rolaq_decode_attn_static(const rolaq_cache* cache, const rolaq_layer_params*
  * The read-side rotation never runs per token: R folds into the absorbed query
  * projection and R^T into the absorbed value projection, so the decode works in the
  * rotated basis and the caller's projections see the original one.  The folded weights
- * are bf16 (computed in fp32, rounded once); every sum runs in fp32.  All pointers are
- * device memory owned by the caller, dense and row-major as listed; fp32 arrays 4-byte,
- * bf16 activations 2-byte and the folded weights 16-byte aligned.  NULL or misaligned
+ * are bf16 (computed in fp32, rounded once).  All pointers are device memory owned by the
+ * caller, dense and row-major as listed; alignment: the folded weights and the per-step
+ * inputs 16 bytes, fp32 arrays otherwise 4 and bf16 outputs 2.  NULL or misaligned
  * pointers, heads <= 0 (or above 65535) and batch < 0 give ROLAQ_EINVAL and launch
  * nothing.  batch == 0 makes the per-step calls a no-op that returns ROLAQ_OK without
  * looking at the pointers (empty tensors may carry NULL).                              */
 
-/* Once per layer: W_q[h] = W_UK[h]^T . R and W_o[h] = R^T . W_UV[h].
+/* Once per layer: W_q[h] = W_UK[h]^T . R and W_o[h] = R^T . W_UV[h] (fp32 sums).
  * W_UK_dev, W_UV_dev fp32 [heads][512][128] (latent row k, head column n: the up
  * projections c . W_UK[h] -> k_nope, c . W_UV[h] -> v); R_dev fp32 [512][512] with
  * y = c . R; W_q_dev bf16 [heads][128][512]; W_o_dev bf16 [heads][512][128].         */
@@ -220,14 +220,16 @@ int rolaq_fold_weights(const float* W_UK_dev, const float* W_UV_dev, const float
 
 /* Per decode step: q_c_rot[b][h] = q_nope[b][h] . W_q[h], the query rolaq_decode_attn
  * takes.  q_nope_dev bf16 [batch][heads][128]; W_q_dev bf16 from rolaq_fold_weights;
- * q_c_rot_dev bf16 [batch][heads][512] (fp32 sum, rounded to nearest even once).     */
+ * q_c_rot_dev bf16 [batch][heads][512].  Tensor-core product of the bf16 operands with
+ * fp32 accumulation, rounded to bf16 (nearest even) once.                            */
 int rolaq_fold_query(const void* q_nope_dev, const void* W_q_dev, int batch, int heads,
                      void* q_c_rot_dev, void* stream);
 
 /* Per decode step: v[b][h] = out[b][h] . W_o[h], the attention output back in the
  * original basis and through the value up-projection.  out_dev fp32 [batch][heads][512]
  * (rolaq_decode_attn's output); W_o_dev bf16 from rolaq_fold_weights; v_dev fp32
- * [batch][heads][128].                                                                */
+ * [batch][heads][128].  out enters the tensor-core product rounded to bf16 (nearest
+ * even); the sums accumulate in fp32.                                                 */
 int rolaq_unfold_output(const float* out_dev, const void* W_o_dev, int batch, int heads,
                         float* v_dev, void* stream);
 
