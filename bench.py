@@ -122,7 +122,7 @@ class DecodeLayer:
         Rm = torch.as_tensor(W.rotation(w.seed + layer)).to(dev)
         self.R_split = R.prepare_rotation(Rm)
         pt = torch.as_tensor(W.page_table(w))
-        self.cache = R.PagedCache(int(pt.max()) + 1, pt, device=dev)
+        self.cache = R.PagedCache(int(pt.max()) + 1, pt, w.n_sink, w.n_recent, device=dev)
         self.q_c = (torch.randn((w.batch, w.heads, W.D_C), device=dev, generator=_gen(w, layer, 7))
                     .to(torch.bfloat16))
         self.q_r = (torch.randn((w.batch, w.heads, W.D_R), device=dev, generator=_gen(w, layer, 8))
@@ -131,6 +131,7 @@ class DecodeLayer:
         self.lse = torch.empty((w.batch, w.heads), dtype=torch.float32, device=dev)
 
     def fill(self, w, layer, dev, chunk=1 << 18):
+        lens = torch.as_tensor(w.seq_lens, dtype=torch.int32, device=dev)   # lengths after the fill
         for b, L in enumerate(w.seq_lens):
             for s in range(0, L, chunk):
                 n = min(chunk, L - s)
@@ -138,7 +139,7 @@ class DecodeLayer:
                 kr = W.rope_key_device(w, layer, n, dev, stream=5000 + 97 * b + s // chunk)
                 req = torch.full((n,), b, dtype=torch.int32, device=dev)
                 pos = torch.arange(s, s + n, dtype=torch.int32, device=dev)
-                R.quantize_append(self.cache, self.params, self.R_split, c, kr, req, pos)
+                R.quantize_append(self.cache, self.params, self.R_split, c, kr, req, pos, lens)
 
 
 def _gen(w, layer, k):
@@ -277,6 +278,7 @@ def run_ours(args, rank, world, dev):
     # prefill write path: 65,536 tokens x 27 layers
     q_stats = bench_quantize(args, dev, world)
     bf16_stats = bench_bf16_baseline(args, dev, world, w, dec_ms)
+    cfg_stats = bench_configs(args, dev)
     proj_stats = [bench_projections(args, dev, world, w.batch, w.heads),
                   bench_projections(args, dev, world, W.PAGED_H128.batch, W.PAGED_H128.heads)]
     clocks = sampler.stop()     # sampled across the timed regions
@@ -305,6 +307,7 @@ def run_ours(args, rank, world, dev):
         "quantize": q_stats,
         "bf16_baseline": bf16_stats,
         "projections": proj_stats,
+        "other_workloads": cfg_stats,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -368,6 +371,68 @@ def capture_graph(fn):
         fn()
     torch.cuda.synchronize()
     return g
+
+
+# ------------------------------------------------------- the other workloads ----
+# Decode on the survey's other decode shapes, each over enough layers that one sweep of
+# the caches exceeds L2 (126 MB): 4 x 32K at 16 heads, 32 requests of log-uniform lengths
+# at 128 heads on shuffled pages, and 64 x 8K with 4 sink + 128 recent bf16 tokens.
+
+def algorithmic_decode_bytes(w):
+    """2-bit tokens at 288 B, protected tokens at 1,152 B (bf16 latent + RoPE key)."""
+    total = 0
+    for L in w.seq_lens:
+        prot = min(L, w.n_sink + w.n_recent) if (w.n_sink or w.n_recent) else 0
+        total += (L - prot) * R.TOKEN_BYTES + prot * R.BF16_TOKEN_BYTES
+    return total
+
+
+def bench_configs(args, dev):
+    hbm, bf16, src = peaks()
+    res = []
+    for w in (W.DECODE_4x32K, W.PAGED_H128, W.MIXED_64x8K):
+        per_layer = algorithmic_decode_bytes(w)
+        nl = max(2, -(-300_000_000 // per_layer))
+        layers = []
+        for l in range(nl):
+            lay = DecodeLayer(w, l, dev)
+            lay.fill(w, l, dev)
+            layers.append(lay)
+        ws = torch.empty(R.decode_workspace_bytes(w.batch, w.heads), dtype=torch.uint8, device=dev)
+        lens = torch.as_tensor(w.seq_lens, dtype=torch.int32, device=dev)
+
+        def sweep():
+            for lay in layers:
+                R.decode_attn(lay.cache, lay.params, lay.q_c, lay.q_r, lens, SM_SCALE, lay.out, lay.lse, ws)
+
+        for _ in range(max(args.warmup, 3)):
+            sweep()
+        torch.cuda.synchronize()
+        assert R.get_status() == 0
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        t0.record()
+        for _ in range(reps):
+            sweep()
+        t1.record()
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / (reps * nl)
+        gbs = per_layer / (ms * 1e-3) / 1e9
+        entry = {"workload": w.name, "batch": w.batch, "heads": w.heads, "tokens": w.total_tokens,
+                 "n_sink": w.n_sink, "n_recent": w.n_recent, "layers_swept": nl,
+                 "bytes_per_layer": per_layer, "ms_per_layer": round(ms, 4),
+                 "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                              "frac": round(gbs / hbm, 4), "frac_of_8tbs": round(gbs / 8000.0, 4),
+                              "peak_source": src}}
+        if w.heads >= 128:
+            flops = 2.0 * w.heads * (R.D_C + R.D_R + R.D_C) * w.total_tokens
+            tf = flops / (ms * 1e-3) / 1e12
+            entry["tensor"] = {"achieved": round(tf, 1), "peak": bf16, "unit": "TFLOP/s",
+                               "frac": round(tf / bf16, 4), "flops_per_layer": flops}
+        res.append(entry)
+        del layers, ws
+        torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------ absorbed projections ----
@@ -473,6 +538,9 @@ def bench_bf16_baseline(args, dev, world, w, dec_ms):
 # output unfold for 32 requests x 128 heads.  They print their own timing.
 
 def run_case(args, dev):
+    if args.case == "configs":
+        print(json.dumps({"case": "configs", "results": bench_configs(args, dev)}), flush=True)
+        return
     if args.case == "decode":
         w = W.Workload("decode_4x128k_h16", 4, (131072,) * 4, 16, seed=4242)
         lay = DecodeLayer(w, 0, dev)
@@ -589,7 +657,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["decode", "quantize", "project"], default=None,
+    ap.add_argument("--case", choices=["decode", "quantize", "project", "configs"], default=None,
                     help="run one small single-kernel case (for ncu captures) instead of the bench")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 1)

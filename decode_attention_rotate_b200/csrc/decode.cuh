@@ -87,21 +87,52 @@ struct DecodeSmem {
 static_assert(sizeof(DecodeSmem) + 1024 <= 227 * 1024, "decode shared memory");
 
 // ---- split plan --------------------------------------------------------------
-// pages_b = ceil(L_b / 64); chunk = max(1, ceil(sum_b pages_b / target)); request b
-// gets ceil(pages_b / chunk) items numbered consecutively in request order.  Executed
-// by one full warp; every lane returns the same values.
+// pages_b = ceil(L_b / 64); chunk = the smallest value >= max(1, ceil(sum_b pages_b /
+// target)) for which the item count sum_b ceil(pages_b / chunk) is at most `target` (one
+// wave of items when `target` is the SM count), or that first value when no chunk fits
+// (more requests than `target`); request b gets ceil(pages_b / chunk) items numbered
+// consecutively in request order.  Executed by one full warp; every lane returns the same
+// values.
 struct PlanInfo { int b, first_page, n_pages, n_items, item_offset, chunk; };
+
+__device__ __forceinline__ int plan_items(const int32_t* seq_lens, int batch, int chunk) {
+    const int lane = threadIdx.x & 31;
+    int items = 0;
+    for (int b = lane; b < batch; b += 32) {
+        const int pages = (max(seq_lens[b], 0) + kPageTok - 1) / kPageTok;
+        items += (pages + chunk - 1) / chunk;
+    }
+    for (int o = 16; o; o >>= 1) items += __shfl_xor_sync(0xffffffffu, items, o);
+    return items;
+}
 
 __device__ __forceinline__ int plan_chunk(const int32_t* seq_lens, int batch, int target) {
     const int lane = threadIdx.x & 31;
     long long total = 0;
+    int max_pages = 0;
     for (int b = lane; b < batch; b += 32) {
-        int L = max(seq_lens[b], 0);
-        total += (L + kPageTok - 1) / kPageTok;
+        const int pages = (max(seq_lens[b], 0) + kPageTok - 1) / kPageTok;
+        total += pages;
+        max_pages = max(max_pages, pages);
     }
-    for (int o = 16; o; o >>= 1) total += __shfl_xor_sync(0xffffffffu, total, o);
-    long long c = (total + target - 1) / target;
-    return (int)max(1LL, c);
+    for (int o = 16; o; o >>= 1) {
+        total += __shfl_xor_sync(0xffffffffu, total, o);
+        max_pages = max(max_pages, __shfl_xor_sync(0xffffffffu, max_pages, o));
+    }
+    int c = (int)max(1LL, (total + target - 1) / target);
+    // ragged lengths can leave more items than `target` (a second, mostly idle wave);
+    // with chunk = max_pages every non-empty request is one item, so when batch <=
+    // target a fitting chunk exists: binary search for the smallest
+    if (batch <= target && max_pages > c && plan_items(seq_lens, batch, c) > target) {
+        int lo = c + 1, hi = max_pages;
+        while (lo < hi) {
+            const int mid = lo + (hi - lo) / 2;
+            if (plan_items(seq_lens, batch, mid) <= target) hi = mid;
+            else lo = mid + 1;
+        }
+        c = lo;
+    }
+    return c;
 }
 
 // Locate work item `item` (or request `req` when item < 0).  n_items = total item count.

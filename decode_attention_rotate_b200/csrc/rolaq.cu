@@ -87,17 +87,18 @@ int check_params(const rolaq_layer_params* p) {
     return ROLAQ_OK;
 }
 
-int decode_target_items(int heads) {
-    const int chunks = heads / 16;
-    return (current_sms() + chunks - 1) / chunks;
+// Split-K target: one work item per SM.  Every 16-head chunk of an item is its own CTA,
+// so with more heads the items run as several waves of equally sized CTAs.
+int decode_target_items() { return current_sms(); }
+
+// Scratch per work item: its partial O and (m, l) for every head.
+size_t decode_item_bytes(int heads) { return (size_t)heads * (ROLAQ_D_C * sizeof(float) + sizeof(float2)); }
+
+size_t decode_ws_bytes_for(int batch, int heads, int target) {
+    return ((size_t)target + (size_t)batch) * decode_item_bytes(heads);
 }
 
-size_t decode_ws_bytes(int batch, int heads) {
-    const size_t items = (size_t)decode_target_items(heads) + (size_t)batch;
-    const size_t o = items * heads * ROLAQ_D_C * sizeof(float);
-    const size_t ml = items * heads * sizeof(float2);
-    return o + ml;
-}
+size_t decode_ws_bytes(int batch, int heads) { return decode_ws_bytes_for(batch, heads, decode_target_items()); }
 
 // Raise a kernel's dynamic shared-memory limit once per device.
 template <typename Kernel>
@@ -230,11 +231,13 @@ size_t rolaq_decode_workspace_bytes(int batch, int heads) {
     return decode_ws_bytes(batch, heads);
 }
 
-int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
-                      const void* q_c_rot_dev, const void* q_R_dev,
-                      const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
-                      float* out_dev, float* lse_dev,
-                      void* workspace_dev, size_t workspace_bytes, void* stream) {
+// The decode with an explicit split-K target (work items before the per-request
+// remainders); the workspace must hold (target + batch) items.
+static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* p,
+                            const void* q_c_rot_dev, const void* q_R_dev,
+                            const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
+                            float* out_dev, float* lse_dev,
+                            void* workspace_dev, size_t workspace_bytes, void* stream, int target) {
     int rc = check_cache(cache);
     if (rc) return rc;
     if ((rc = check_params(p))) return rc;
@@ -245,7 +248,8 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
         !aligned(out_dev, 16) || !aligned(workspace_dev, 16) || (lse_dev && !aligned(lse_dev, 4)))
         return ROLAQ_EINVAL;
     if (!isfinite(sm_scale)) return ROLAQ_EINVAL;
-    if (workspace_bytes < decode_ws_bytes(batch, heads)) return ROLAQ_ENOSPACE;
+    if (target < 1) return ROLAQ_ENOSPACE;
+    if (workspace_bytes < decode_ws_bytes_for(batch, heads, target)) return ROLAQ_ENOSPACE;
 
     // The pool as rows of 128 B; one box is a whole page (144 rows).
     CUtensorMap map_page;
@@ -254,7 +258,6 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
                    ROLAQ_PAGE_BYTES / 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return ROLAQ_ECUDA;
 
-    const int target = decode_target_items(heads);
     const int items_cap = target + batch;
     DecodeArgs a;
     a.page_table = cache->page_table_dev;
@@ -285,6 +288,15 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
     rolaq_decode_merge<<<dim3(batch, heads), kMergeThreads, 0, s>>>(a.ws_o, a.ws_ml, seq_lens_dev, batch, heads,
                                                          target, out_dev, lse_dev);
     return launch_status();
+}
+
+int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
+                      const void* q_c_rot_dev, const void* q_R_dev,
+                      const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
+                      float* out_dev, float* lse_dev,
+                      void* workspace_dev, size_t workspace_bytes, void* stream) {
+    return decode_attn_impl(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale, out_dev,
+                            lse_dev, workspace_dev, workspace_bytes, stream, decode_target_items());
 }
 
 // ---- decode with library-owned scratch -------------------------------------------
@@ -318,13 +330,16 @@ int rolaq_decode_attn_static(const rolaq_cache* cache, const rolaq_layer_params*
                              float* out_dev, float* lse_dev, void* stream) {
     if (heads <= 0 || heads % 16) return ROLAQ_EUNSUPPORTED;
     if (batch <= 0) return ROLAQ_EINVAL;
-    if (decode_ws_bytes(batch, heads) > (size_t)ROLAQ_STATIC_SCRATCH_BYTES) return ROLAQ_ENOSPACE;
+    // as many split-K items as the fixed array holds, up to one per SM
+    const long long fit = (long long)(ROLAQ_STATIC_SCRATCH_BYTES / decode_item_bytes(heads)) - batch;
+    const int target = (int)(fit < decode_target_items() ? fit : decode_target_items());
+    if (target < 1) return ROLAQ_ENOSPACE;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ROLAQ_ECUDA;
     void* scratch = static_scratch_ptr(dev);
     if (!scratch) return ROLAQ_ECUDA;
-    return rolaq_decode_attn(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale,
-                             out_dev, lse_dev, scratch, (size_t)ROLAQ_STATIC_SCRATCH_BYTES, stream);
+    return decode_attn_impl(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale, out_dev,
+                            lse_dev, scratch, (size_t)ROLAQ_STATIC_SCRATCH_BYTES, stream, target);
 }
 
 int rolaq_fold_weights(const float* W_UK_dev, const float* W_UV_dev, const float* R_dev,

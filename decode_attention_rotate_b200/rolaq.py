@@ -23,6 +23,7 @@ D_V = 128               # per-head value width
 PAGE_TOKENS = 64
 PAGE_BYTES = 18432
 TOKEN_BYTES = 288
+BF16_TOKEN_BYTES = 1152   # uncompressed MLA record: (512 + 64) x bf16
 RSPLIT_BYTES = 3 * 512 * 512 * 2
 
 STATUS_BAD_PAGE = 1

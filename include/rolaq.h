@@ -151,7 +151,9 @@ int rolaq_quantize_append(const rolaq_cache* cache, const rolaq_layer_params* p,
                           const int32_t* seq_lens_dev, int n, void* stream);
 
 /* Bytes of device workspace rolaq_decode_attn needs for `batch` requests and `heads`
- * query heads on the current device (split-K partials and their merge state).          */
+ * query heads on the current device (split-K partials and their merge state):
+ * (SM count + batch) x heads x 2,056 bytes; 0 for batch <= 0 or heads not a positive
+ * multiple of 16.                                                                      */
 size_t rolaq_decode_workspace_bytes(int batch, int heads);
 
 /* Read path [S2.1], [S3.3]: absorbed-MLA decode attention straight from the packed cache.
@@ -187,8 +189,9 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
  * allocation after start-up.  The call itself allocates nothing.
  *   - The first call on each device looks up the array's device address on that device;
  *     make that first call before any stream capture.
- *   - Requests whose scratch would exceed ROLAQ_STATIC_SCRATCH_BYTES (that is,
- *     rolaq_decode_workspace_bytes(batch, heads) > ROLAQ_STATIC_SCRATCH_BYTES) return
+ *   - The split-K plan uses as many work items as the array holds, up to one per SM:
+ *     (items + batch) x heads x 2,056 bytes <= ROLAQ_STATIC_SCRATCH_BYTES.  A call for
+ *     which not even one item fits ((1 + batch) x heads x 2,056 bytes above it) returns
  *     ROLAQ_ENOSPACE before anything is launched.
  *   - Every call on a device shares the one array and leaves its contents behind; the
  *     kernels overwrite whatever they read, so nothing needs clearing, but calls that can
