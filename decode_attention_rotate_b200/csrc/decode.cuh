@@ -32,16 +32,17 @@ namespace rolaq {
 constexpr int kPageTok = ROLAQ_PAGE_TOKENS;
 constexpr int kPageRows = ROLAQ_PAGE_BYTES / 128;   // 144 rows of 128 B
 constexpr int kDecodeThreads = 512;
-constexpr int kStages = 3;                          // pages in flight
+// HC = query heads per CTA (16 or 32): the N of both tensor-core products.
+template <int HC> __host__ __device__ constexpr int stages_for() { return HC == 16 ? 3 : 2; }   // pages in flight
 constexpr int kSoftWarp0 = 4;                       // softmax warps 4..7 (TMEM lane quarters)
 constexpr int kDqWarp0 = 8;                         // dequant warps 8..15
 constexpr int kXAtom = kPageTok * 128;              // one 64-channel column block of an x tile
 constexpr int kXTile = 8 * kXAtom;                  // 64 KB: 64 tokens x 512 fp16
 constexpr int kMetaRow = 64;                        // page rows: codes 0..63, meta 64..79,
 constexpr int kKrRow = 80;                          // RoPE keys 80..143
-constexpr int kSCol = 0;                            // TMEM: S tiles at columns 0 and 16
-constexpr int kOCol = 64;                           //       O at 64..127 (16 per group)
-constexpr int kTmemCols = 128;
+constexpr int kSCol = 0;                            // TMEM: S tiles at columns 0 and HC
+constexpr int kOCol = 64;                           //       O at 64.. (HC per group)
+template <int HC> __host__ __device__ constexpr int tmem_cols_for() { return HC == 16 ? 128 : 256; }
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kF16Max = 65504.f;
 
@@ -62,15 +63,17 @@ struct DecodeArgs {
     float2* ws_ml;               // [items][heads]       (m (log2 units), sum_t 2^(s_t - m))
 };
 
+template <int HC>
 struct DecodeSmem {
+    static constexpr int kStages = stages_for<HC>();
     alignas(1024) uint8_t x[2][kXTile];                   // x tiles (K-major, 128-byte swizzle)
     alignas(1024) uint8_t stage[kStages][ROLAQ_PAGE_BYTES];
-    alignas(128) uint8_t qc[16 * ROLAQ_D_C * 2];          // fp16 query, QK B operand
-    alignas(128) uint8_t qr[16 * ROLAQ_D_R * 2];          // bf16 RoPE query, B operand
-    alignas(128) uint8_t P[2][16 * kPageTok * 2];         // fp16 probabilities, PV B operand
-    float red[4][16];                                     // softmax warps: per-warp head values
-    float mref[16];                                       // running reference max per head
-    float alpha[16];                                      // its last rescale factor
+    alignas(128) uint8_t qc[HC * ROLAQ_D_C * 2];          // fp16 query, QK B operand
+    alignas(128) uint8_t qr[HC * ROLAQ_D_R * 2];          // bf16 RoPE query, B operand
+    alignas(128) uint8_t P[2][HC * kPageTok * 2];         // fp16 probabilities, PV B operand
+    float red[4][HC];                                     // softmax warps: per-warp head values
+    float mref[HC];                                       // running reference max per head
+    float alpha[HC];                                      // its last rescale factor
     int vote[2][4];
     alignas(8) uint64_t full[kStages];     // page copy landed
     alignas(8) uint64_t pfree[kStages];    // page read by the dequant warps and the QK MMAs
@@ -84,7 +87,8 @@ struct DecodeSmem {
     int plan[4];
     int abort;
 };
-static_assert(sizeof(DecodeSmem) + 1024 <= 227 * 1024, "decode shared memory");
+static_assert(sizeof(DecodeSmem<16>) + 1024 <= 227 * 1024, "decode shared memory (16 heads)");
+static_assert(sizeof(DecodeSmem<32>) + 1024 <= 227 * 1024, "decode shared memory (32 heads)");
 
 // ---- split plan --------------------------------------------------------------
 // pages_b = ceil(L_b / 64); chunk = the smallest value >= max(1, ceil(sum_b pages_b /
@@ -204,10 +208,12 @@ __device__ __forceinline__ void dequant_word2(uint32_t w, uint2 la, uint2 lb, ui
 }
 
 // ---- tensor-core operands -----------------------------------------------------
-// Instruction descriptors: fp32 accumulate, K-major unless noted, N = 16 heads.
-constexpr uint32_t kIdQk = (1u << 4) | ((16u >> 3) << 17) | ((64u >> 4) << 24);                 // f16, M = 64
-constexpr uint32_t kIdRope = kIdQk | (1u << 7) | (1u << 10);                                     // bf16, M = 64
-constexpr uint32_t kIdPv = (1u << 4) | (1u << 15) | ((16u >> 3) << 17) | ((128u >> 4) << 24);   // f16, M = 128, A MN-major
+// Instruction descriptors: fp32 accumulate, K-major unless noted, N = HC heads.
+template <int HC> __host__ __device__ constexpr uint32_t id_qk() { return (1u << 4) | ((uint32_t)(HC >> 3) << 17) | ((64u >> 4) << 24); }  // f16, M = 64
+template <int HC> __host__ __device__ constexpr uint32_t id_rope() { return id_qk<HC>() | (1u << 7) | (1u << 10); }                      // bf16, M = 64
+template <int HC> __host__ __device__ constexpr uint32_t id_pv() {                                                                      // f16, M = 128, A MN-major
+    return (1u << 4) | (1u << 15) | ((uint32_t)(HC >> 3) << 17) | ((128u >> 4) << 24);
+}
 
 // Column slot of channel order inside every 16-channel block: the PRMT lookup yields the
 // pairs (k, k+4), so slot 2k + e of a block of 8 holds channel k + 4e.  The query is laid
@@ -235,9 +241,10 @@ __device__ __forceinline__ bool page_ok(const DecodeArgs& args, long long pid) {
 }
 // Issue the bulk copy of one page (all 144 rows) into stage k % kStages, or mark the
 // stage invalid when the page-table entry is outside the pool.
-__device__ __forceinline__ void load_page(DecodeSmem& sm, const CUtensorMap* map, const DecodeArgs& args,
+template <int HC>
+__device__ __forceinline__ void load_page(DecodeSmem<HC>& sm, const CUtensorMap* map, const DecodeArgs& args,
                                           long long pid, int k) {
-    const int st = k % kStages;
+    const int st = k % DecodeSmem<HC>::kStages;
     const uint32_t bar = smem_u32(&sm.full[st]);
     if (page_ok(args, pid)) {
         sm.valid[st] = 1;
@@ -309,14 +316,34 @@ __device__ __forceinline__ void store_tile_part(uint8_t* xt, int t, int g, const
     }
 }
 
+// Scores of one softmax warp: 16 TMEM lanes x HC columns (16x256b shape, HC / 8 repeats).
+__device__ __forceinline__ void tmem_ld_scores(uint32_t taddr, uint32_t (&u)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_scores(uint32_t taddr, uint32_t (&u)[16]) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+                   "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]),
+                   "=r"(u[15])
+                 : "r"(taddr));
+}
+
+template <int HC>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
 rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArgs args) {
     extern __shared__ uint8_t smem_raw[];
+    constexpr int kStages = DecodeSmem<HC>::kStages;
+    constexpr int kTmemCols = tmem_cols_for<HC>();
+    constexpr uint32_t kIdQk = id_qk<HC>(), kIdRope = id_rope<HC>(), kIdPv = id_pv<HC>();
     // offset the __shared__ array itself (not an integer address) so that every access
     // stays a shared-memory access
-    DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
+    DecodeSmem<HC>& sm =
+        *reinterpret_cast<DecodeSmem<HC>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int hc = blockIdx.y;                 // 16-head chunk
+    const int hc = blockIdx.y;                 // HC-head chunk
 
     if (warp == 0) {
         PlanInfo pi = plan_lookup(args.seq_lens, args.batch, args.target_items, (int)blockIdx.x, -1);
@@ -340,7 +367,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             mbar_init(smem_u32(&sm.sfree[s]), 4);
             mbar_init(smem_u32(&sm.pready[s]), 4);
         }
-        for (int h = 0; h < 16; ++h) sm.mref[h] = -INFINITY;
+        for (int h = 0; h < HC; ++h) sm.mref[h] = -INFINITY;
         sm.abort = 0;
         fence_mbar_init();
         prefetch_tmap(&map_page);
@@ -350,7 +377,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
     if (b < 0) return;                         // item past the end of the plan
     const int first_page = sm.plan[1], T = sm.plan[2];
     const int L = args.seq_lens[b];
-    const int h0 = hc * 16;
+    const int h0 = hc * HC;
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      :: "r"(smem_u32(&sm.tmem_base)), "r"(kTmemCols) : "memory");
@@ -360,7 +387,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
     {
         const uint16_t* qb = reinterpret_cast<const uint16_t*>(args.q + ((size_t)b * args.heads + h0) * ROLAQ_D_C);
         float qmax = 0.f;
-        for (int e = threadIdx.x; e < 16 * ROLAQ_D_C / 2; e += kDecodeThreads) {
+        for (int e = threadIdx.x; e < HC * ROLAQ_D_C / 2; e += kDecodeThreads) {
             const int n = e / (ROLAQ_D_C / 2), s = 2 * (e % (ROLAQ_D_C / 2));
             const float v0 = __uint_as_float((uint32_t)qb[n * ROLAQ_D_C + slot_channel(s)] << 16);
             const float v1 = __uint_as_float((uint32_t)qb[n * ROLAQ_D_C + slot_channel(s + 1)] << 16);
@@ -369,7 +396,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
         }
         if (!(qmax < kF16Max)) raise_status(ROLAQ_STATUS_RANGE);
         const uint32_t* rb = reinterpret_cast<const uint32_t*>(args.qr + ((size_t)b * args.heads + h0) * ROLAQ_D_R);
-        for (int e = threadIdx.x; e < 16 * ROLAQ_D_R / 2; e += kDecodeThreads) {
+        for (int e = threadIdx.x; e < HC * ROLAQ_D_R / 2; e += kDecodeThreads) {
             const int n = e / (ROLAQ_D_R / 2), k = 2 * (e % (ROLAQ_D_R / 2));
             *reinterpret_cast<uint32_t*>(sm.qr + plain_off(n, k, 8 * 128)) = rb[e];
         }
@@ -416,7 +443,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                     for (int g = 0; g < 4; ++g) {
 #pragma unroll
                         for (int ks = 0; ks < kPageTok / 16; ++ks)
-                            umma_ss1(tmem + kOCol + 16 * g, da + (uint64_t)((2 * g * kXAtom + ks * 2048) >> 4),
+                            umma_ss1(tmem + kOCol + HC * g, da + (uint64_t)((2 * g * kXAtom + ks * 2048) >> 4),
                                      db + (uint64_t)((ks * 256) >> 4), kIdPv, ks > 0 ? 1u : first);
                         if (g == 1) umma_commit(smem_u32(&sm.xfree[bj][0]));   // groups 0-1 read
                     }
@@ -429,7 +456,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                 if (i >= 2) mbar_wait(smem_u32(&sm.sfree[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
                 const uint64_t da = dxk + (uint64_t)(bi * (kXTile >> 4));
                 const uint64_t dk = dkr + (uint64_t)(st * (ROLAQ_PAGE_BYTES >> 4));
-                const uint32_t d = tmem + kSCol + 16 * bi;
+                const uint32_t d = tmem + kSCol + HC * bi;
                 // channel groups 0-1 (K steps 0..15) as soon as that half of the tile is written
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
@@ -491,15 +518,18 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
         // ------------------------------------------------------------- softmax ----
         // Warp q reads TMEM lane quarter q: S rows 16q..16q+15 (M = 64) in lanes 0..15 with
         // the 16x256b shape, so lane (r, i) holds rows 16q + r and 16q + r + 8 of heads
-        // 2i, 2i+1, 8+2i, 9+2i; O rows (slots) 32q..32q+31 of every group.
+        // 8k + 2i and 8k + 2i + 1 (k < HC / 8); O rows (slots) 32q..32q+31 of every group.
+        constexpr int kE = HC / 4;             // heads per thread
         const int q = warp - kSoftWarp0;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const int r = lane >> 2, i4 = lane & 3;
         const int rows[2] = {16 * q + r, 16 * q + r + 8};
-        const int heads[4] = {2 * i4, 2 * i4 + 1, 8 + 2 * i4, 9 + 2 * i4};
-        float m_ref[4], l[4];
+        int heads[kE];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) { m_ref[e] = -INFINITY; l[e] = 0.f; }
+        for (int e = 0; e < kE; ++e) heads[e] = 8 * (e >> 1) + 2 * i4 + (e & 1);
+        float m_ref[kE], l[kE];
+#pragma unroll
+        for (int e = 0; e < kE; ++e) { m_ref[e] = -INFINITY; l[e] = 0.f; }
         long long pid_next = page_id(args, b, page_of(0));
         for (int i = 0; i < T; ++i) {
             const int bi = i & 1;
@@ -508,23 +538,20 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             mbar_wait(smem_u32(&sm.sfull[bi]), (unsigned)((i >> 1) & 1), &sm.abort);
             __syncwarp();
             tc_fence_after();
-            uint32_t u[8];
-            asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
-                           "=r"(u[7])
-                         : "r"(tmem + lane_base + kSCol + 16 * bi));
+            uint32_t u[HC / 2];
+            tmem_ld_scores(tmem + lane_base + kSCol + HC * bi, u);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.sfree[bi]));
             // s[e][j]: head heads[e], row rows[j]
-            float s2[4][2];
+            float s2[kE][2];
             bool up = false;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const bool valid = vpage && page_of(i) * kPageTok + rows[j] < L;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
+                for (int e = 0; e < kE; ++e) {
                     const uint32_t raw = u[(e >> 1) * 4 + 2 * j + (e & 1)];
                     s2[e][j] = valid ? __uint_as_float(raw) * args.scale_log2 : -INFINITY;
                     up |= s2[e][j] > m_ref[e] + kRescaleLog2 || (m_ref[e] == -INFINITY && s2[e][j] > -INFINITY);
@@ -538,7 +565,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             if (any) {
                 // per-head max over the tile: lanes sharing i4 hold the same heads
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
+                for (int e = 0; e < kE; ++e) {
                     float mx = fmaxf(s2[e][0], s2[e][1]);
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -546,7 +573,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                     if (r == 0) sm.red[q][heads[e]] = mx;
                 }
                 named_bar_sync(1, 128);
-                if (q == 0 && lane < 16) {
+                if (q == 0 && lane < HC) {
                     // one thread per head: new reference and factor for all warps
                     const int h = lane;
                     const float tm = fmaxf(fmaxf(sm.red[0][h], sm.red[1][h]), fmaxf(sm.red[2][h], sm.red[3][h]));
@@ -562,26 +589,27 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                 named_bar_sync(1, 128);
                 bool moved = false;
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
+                for (int e = 0; e < kE; ++e) {
                     const float al = sm.alpha[heads[e]];
                     m_ref[e] = sm.mref[heads[e]];
                     l[e] *= al;
                 }
 #pragma unroll
-                for (int h = 0; h < 16; ++h) moved |= sm.alpha[h] != 1.f;
+                for (int h = 0; h < HC; ++h) moved |= sm.alpha[h] != 1.f;
                 if (moved && i > 0) {
                     // O holds PV of tiles 0..i-1: wait for PV(i-1), scale this quarter's lanes
                     mbar_wait(smem_u32(&sm.xfree[(i - 1) & 1][1]), (unsigned)(((i - 1) >> 1) & 1), &sm.abort);
                     __syncwarp();
                     tc_fence_after();
 #pragma unroll 1
-                    for (int g = 0; g < 4; ++g) {
+                    for (int gc = 0; gc < 4 * (HC / 16); ++gc) {       // 16-column slices of O
                         uint32_t v[16];
-                        tmem_ld16(tmem + lane_base + kOCol + 16 * g, v);
+                        tmem_ld16(tmem + lane_base + kOCol + 16 * gc, v);
                         tmem_ld_wait();
+                        const int hb = 16 * (gc % (HC / 16));            // first head of the slice
 #pragma unroll
-                        for (int h = 0; h < 16; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * sm.alpha[h]);
-                        tmem_st16(tmem + lane_base + kOCol + 16 * g, v);
+                        for (int h = 0; h < 16; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * sm.alpha[hb + h]);
+                        tmem_st16(tmem + lane_base + kOCol + 16 * gc, v);
                     }
                     tmem_st_wait();
                     tc_fence_before();
@@ -592,7 +620,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             if (i >= 2) mbar_wait(smem_u32(&sm.xfree[bi][1]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
             uint8_t* P = sm.P[bi];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
+            for (int e = 0; e < kE; ++e)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const float p = (m_ref[e] == -INFINITY) ? 0.f : ex2(s2[e][j] - m_ref[e]);
@@ -609,17 +637,18 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
         tc_fence_after();
         const int m = 32 * q + lane;           // O row = slot within the group
 #pragma unroll 1
-        for (int g = 0; g < 4; ++g) {
+        for (int gc = 0; gc < 4 * (HC / 16); ++gc) {           // 16-column slices of O
+            const int g = gc / (HC / 16), hb = 16 * (gc % (HC / 16));
             uint32_t v[16];
-            tmem_ld16(tmem + lane_base + kOCol + 16 * g, v);
+            tmem_ld16(tmem + lane_base + kOCol + 16 * gc, v);
             tmem_ld_wait();
-            float* dst = args.ws_o + ((size_t)blockIdx.x * args.heads + h0) * ROLAQ_D_C + 128 * g + slot_channel(m);
+            float* dst = args.ws_o + ((size_t)blockIdx.x * args.heads + h0 + hb) * ROLAQ_D_C + 128 * g + slot_channel(m);
 #pragma unroll
             for (int h = 0; h < 16; ++h) dst[(size_t)h * ROLAQ_D_C] = __uint_as_float(v[h]);
         }
         // row sums: lanes sharing i4 (8 per warp) and the four warps
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int e = 0; e < kE; ++e) {
             float v = l[e];
             v += __shfl_xor_sync(0xffffffffu, v, 4);
             v += __shfl_xor_sync(0xffffffffu, v, 8);
@@ -627,7 +656,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             if (r == 0) sm.red[q][heads[e]] = v;
         }
         named_bar_sync(1, 128);
-        if (q == 0 && lane < 16) {
+        if (q == 0 && lane < HC) {
             const int h = lane;
             args.ws_ml[(size_t)blockIdx.x * args.heads + h0 + h] =
                 make_float2(sm.mref[h], (sm.red[0][h] + sm.red[1][h]) + (sm.red[2][h] + sm.red[3][h]));

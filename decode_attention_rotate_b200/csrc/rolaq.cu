@@ -279,11 +279,20 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
     a.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace_dev) +
                                         (size_t)items_cap * heads * ROLAQ_D_C * sizeof(float));
 
-    const size_t smem = sizeof(DecodeSmem) + 1024;
-    static bool attr_done[kMaxDevices] = {false};
-    set_smem_limit_once(rolaq_decode_split, smem, attr_done);
+    // 32 heads per CTA when the head count allows it (twice the work per tensor-core
+    // instruction and per dequantised tile), else 16
     cudaStream_t s = (cudaStream_t)stream;
-    rolaq_decode_split<<<dim3(items_cap, heads / 16), kDecodeThreads, smem, s>>>(map_page, a);
+    if (heads % 32 == 0) {
+        const size_t smem = sizeof(DecodeSmem<32>) + 1024;
+        static bool attr_done[kMaxDevices] = {false};
+        set_smem_limit_once(rolaq_decode_split<32>, smem, attr_done);
+        rolaq_decode_split<32><<<dim3(items_cap, heads / 32), kDecodeThreads, smem, s>>>(map_page, a);
+    } else {
+        const size_t smem = sizeof(DecodeSmem<16>) + 1024;
+        static bool attr_done[kMaxDevices] = {false};
+        set_smem_limit_once(rolaq_decode_split<16>, smem, attr_done);
+        rolaq_decode_split<16><<<dim3(items_cap, heads / 16), kDecodeThreads, smem, s>>>(map_page, a);
+    }
     if ((rc = launch_status())) return rc;
     rolaq_decode_merge<<<dim3(batch, heads), kMergeThreads, 0, s>>>(a.ws_o, a.ws_ml, seq_lens_dev, batch, heads,
                                                          target, out_dev, lse_dev);

@@ -225,6 +225,13 @@ def test_decode_128_heads_paged():
     _decode_case(w, [1024, 2500, 64, 1500], 128, 0.88, 1.02)
 
 
+@pytest.mark.parametrize("H", [32, 48, 64])
+def test_decode_head_counts(H):
+    # 32 and 64 heads take 32-head CTAs, 48 heads three 16-head CTAs per work item
+    w = W.Workload("hc%d" % H, 3, (700, 64, 1999), H, paged_shuffled=True, seed=97 + H)
+    _decode_case(w, [700, 64, 1999], H, 0.93, 1.08, n_sink=4, n_recent=64)
+
+
 def test_decode_sink_and_recent_protection():
     w = W.Workload("mix", 3, (1000, 130, 5), 16, seed=93)
     _decode_case(w, [1000, 130, 5], 16, 0.97, 1.1, n_sink=4, n_recent=128)
