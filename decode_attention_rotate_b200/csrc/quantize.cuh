@@ -240,42 +240,55 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
         // ----------------------------------------------------------------- MMA ----
         // Chain A (TMEM columns buf*256 .. +127): R_lo and R_mid over all of K, then R_hi
         // over K < 256.  Chain B (+128 .. +255): R_hi over K >= 256.  y = A + B.
-        if (lane == 0) {
+        // The whole warp runs the loop (waits and descriptors are warp-uniform, so the
+        // operands stay in uniform registers); one elected lane issues each chunk's MMAs
+        // and commits.
+        {
             uint32_t it = 0, job = 0;
             int tl = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tl)
                 for (int g = 0; g < ROLAQ_GROUPS && ok; ++g, ++job) {
                     const uint32_t buf = job & 1, use = job >> 1;
-                    if (use >= 1 && !mbar_wait(smem_u32(&sm.tempty[buf]), (use - 1) & 1, &sm.abort)) { ok = false; break; }
+                    if (use >= 1)
+                        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.tempty[buf]), (use - 1) & 1, &sm.abort));
+                    if (!ok) break;
                     tc_fence_after();
                     const uint32_t d_a = tmem + buf * 2 * kQN, d_b = d_a + kQN;
                     for (int pass = 0; pass < 2 && ok; ++pass)
                         for (int kc = 0; kc < kQKSteps; ++kc, ++it) {
-                            if (g == 0 && pass == 0 &&
-                                !mbar_wait(smem_u32(&sm.a_full[kc]), tl & 1, &sm.abort)) { ok = false; break; }
+                            if (g == 0 && pass == 0)
+                                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.a_full[kc]), tl & 1, &sm.abort));
                             const int st = it % kQStages;
-                            if (!mbar_wait(smem_u32(&sm.full[st]), (it / kQStages) & 1, &sm.abort)) { ok = false; break; }
+                            if (ok)
+                                ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.full[st]), (it / kQStages) & 1, &sm.abort));
+                            if (!ok) break;
                             tc_fence_after();
                             const uint32_t sa = smem_u32(sm.a[kc]);
                             const uint32_t sb0 = smem_u32(sm.b[st][0]), sb1 = smem_u32(sm.b[st][1]);
+                            if (elect_one()) {
 #pragma unroll
-                            for (int k16 = 0; k16 < 2; ++k16) {
-                                const uint64_t da = umma_desc_sw64(sa + 32 * k16);
-                                const uint64_t db0 = umma_desc_sw64(sb0 + 32 * k16);
-                                if (pass == 0) {
-                                    umma_bf16(d_a, da, db0, (kc | k16) != 0);
-                                    umma_bf16(d_a, da, umma_desc_sw64(sb1 + 32 * k16), 1u);
-                                } else if (kc < kQKSteps / 2) {
-                                    umma_bf16(d_a, da, db0, 1u);
-                                } else {
-                                    umma_bf16(d_b, da, db0, (kc > kQKSteps / 2 || k16 > 0) ? 1u : 0u);
+                                for (int k16 = 0; k16 < 2; ++k16) {
+                                    const uint64_t da = umma_desc_sw64(sa + 32 * k16);
+                                    const uint64_t db0 = umma_desc_sw64(sb0 + 32 * k16);
+                                    if (pass == 0) {
+                                        umma_bf16(d_a, da, db0, (kc | k16) != 0);
+                                        umma_bf16(d_a, da, umma_desc_sw64(sb1 + 32 * k16), 1u);
+                                    } else if (kc < kQKSteps / 2) {
+                                        umma_bf16(d_a, da, db0, 1u);
+                                    } else {
+                                        umma_bf16(d_b, da, db0, (kc > kQKSteps / 2 || k16 > 0) ? 1u : 0u);
+                                    }
                                 }
+                                umma_commit(smem_u32(&sm.empty[st]));
+                                if (g == ROLAQ_GROUPS - 1 && pass == 1) umma_commit(smem_u32(&sm.a_free[kc]));
                             }
-                            umma_commit(smem_u32(&sm.empty[st]));
-                            if (g == ROLAQ_GROUPS - 1 && pass == 1) umma_commit(smem_u32(&sm.a_free[kc]));
+                            __syncwarp();
                         }
-                    if (ok) umma_commit(smem_u32(&sm.tfull[buf]));
+                    if (ok) {
+                        if (elect_one()) umma_commit(smem_u32(&sm.tfull[buf]));
+                        __syncwarp();
+                    }
                 }
         }
     } else {
@@ -396,6 +409,11 @@ rolaq_quantize_small_kernel(const __nv_bfloat16* __restrict__ R_split, const __n
     __shared__ float s_y[kSmallTok][ROLAQ_GROUP];
     __shared__ float s_red[4];
     __shared__ uint32_t s_codes[kSmallTok][8];
+    // each token's target, looked up before the dot products so that the dependent
+    // global loads (request, position, page table, length) overlap them
+    __shared__ long long s_pid[kSmallTok], s_prow[kSmallTok];
+    __shared__ int s_row[kSmallTok];
+    __shared__ __align__(16) uint2 s_kr[kSmallTok][ROLAQ_KR_BYTES / 8];
     const uint32_t rank = cluster_ctarank();     // output slice of the group
     const int g = blockIdx.y;                    // group
     const int t0 = blockIdx.z * kSmallTok;
@@ -408,6 +426,29 @@ rolaq_quantize_small_kernel(const __nv_bfloat16* __restrict__ R_split, const __n
         reinterpret_cast<uint4*>(s_c[t])[k8] = v;
     }
     if (threadIdx.x < kSmallTok * 8) s_codes[threadIdx.x >> 3][threadIdx.x & 7] = 0;
+    if (rank == 0 && threadIdx.x < nt) {
+        const int t = threadIdx.x, tok = t0 + t;
+        const int rq = args.req[tok], ps = args.pos[tok];
+        long long pid = -1, prow = -1;
+        if (rq >= 0 && rq < args.batch && ps >= 0 && (ps / ROLAQ_PAGE_TOKENS) < args.max_pages) {
+            pid = args.page_table[(long long)rq * args.max_pages + ps / ROLAQ_PAGE_TOKENS];
+            if (pid >= args.num_pages) pid = -1;
+        }
+        if (pid >= 0 && args.prot) {
+            const int nslot = args.n_sink + args.n_recent;
+            if (ps < args.n_sink)
+                prow = (long long)rq * nslot + ps;
+            else if (args.n_recent > 0 && ps >= args.seq_lens[rq] - args.n_recent)
+                prow = (long long)rq * nslot + args.n_sink + ps % args.n_recent;
+        }
+        s_pid[t] = pid;
+        s_prow[t] = prow;
+        s_row[t] = ps % ROLAQ_PAGE_TOKENS;
+    }
+    if (rank == 0 && g == 0 && threadIdx.x >= 128 && threadIdx.x < 128 + kSmallTok * 16) {
+        const int t = (threadIdx.x - 128) >> 4, j = threadIdx.x & 15;
+        if (t < nt) s_kr[t][j] = reinterpret_cast<const uint2*>(args.k_r + (size_t)(t0 + t) * ROLAQ_D_R)[j];
+    }
     __syncthreads();
     cluster_sync();                              // every CTA of the cluster is running
     const uint32_t y_first = mapa_shared(smem_u32(&s_y[0][0]), 0);
@@ -454,7 +495,6 @@ rolaq_quantize_small_kernel(const __nv_bfloat16* __restrict__ R_split, const __n
     if (threadIdx.x >= ROLAQ_GROUP) return;      // warps 0..3 finish the group
     const int j = threadIdx.x;
     for (int t = 0; t < nt; ++t) {
-        const int tok = t0 + t;
         const float y = s_y[t][j];
         const float mean = block_sum128(y, s_red) * (1.f / 128.f);
         const float d = y - mean;
@@ -463,36 +503,22 @@ rolaq_quantize_small_kernel(const __nv_bfloat16* __restrict__ R_split, const __n
         const float z = d * inv;
         const uint32_t code = (uint32_t)(z >= -args.tau) + (uint32_t)(z >= 0.f) + (uint32_t)(z >= args.tau);
         atomicOr(&s_codes[t][j >> 4], code << (2 * (j & 15)));
-        const int rq = args.req[tok], ps = args.pos[tok];
-        long long pid = -1;
-        if (rq >= 0 && rq < args.batch && ps >= 0 && (ps / ROLAQ_PAGE_TOKENS) < args.max_pages) {
-            pid = args.page_table[(long long)rq * args.max_pages + ps / ROLAQ_PAGE_TOKENS];
-            if (pid >= args.num_pages) pid = -1;
-        }
+        const long long pid = s_pid[t];
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (pid < 0) {
             if (j == 0 && g == 0) raise_status(ROLAQ_STATUS_BAD_SLOT);
             continue;
         }
         uint8_t* page = args.pages + pid * (long long)ROLAQ_PAGE_BYTES;
-        const int row = ps % ROLAQ_PAGE_TOKENS;
+        const int row = s_row[t];
         if (j < 8)
             reinterpret_cast<uint32_t*>(page + ROLAQ_PAGE_CODES_OFFSET + row * ROLAQ_CODE_BYTES + 32 * g)[j] = s_codes[t][j];
         if (j == 0)
             *reinterpret_cast<float2*>(page + ROLAQ_PAGE_META_OFFSET + row * ROLAQ_META_BYTES + 8 * g) =
                 make_float2(mean, args.gain * sd);
-        if (g == 0 && j < 16)
-            reinterpret_cast<uint2*>(page + ROLAQ_PAGE_KR_OFFSET + row * ROLAQ_KR_BYTES)[j] =
-                reinterpret_cast<const uint2*>(args.k_r + (size_t)tok * ROLAQ_D_R)[j];
-        if (args.prot) {
-            const int nslot = args.n_sink + args.n_recent;
-            long long prow = -1;
-            if (ps < args.n_sink)
-                prow = (long long)rq * nslot + ps;
-            else if (args.n_recent > 0 && ps >= args.seq_lens[rq] - args.n_recent)
-                prow = (long long)rq * nslot + args.n_sink + ps % args.n_recent;
-            if (prow >= 0) args.prot[prow * ROLAQ_D_C + 128 * g + j] = __float2bfloat16_rn(y);
-        }
+        if (g == 0 && j < 16) reinterpret_cast<uint2*>(page + ROLAQ_PAGE_KR_OFFSET + row * ROLAQ_KR_BYTES)[j] = s_kr[t][j];
+        const long long prow = s_prow[t];
+        if (prow >= 0) args.prot[prow * ROLAQ_D_C + 128 * g + j] = __float2bfloat16_rn(y);
     }
 }
 
