@@ -35,10 +35,10 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 # DRAM bytes (read + write) of the split kernel per decode launch of the bench workload,
 # from the ncu capture summarised in profiles/decode_split_4x128k_h16.md (4 x 131,072
-# tokens): the 151.23 MB of reads scale with the tokens (x2 here); the 3.87 MB of split-K
+# tokens): the 151.18 MB of reads scale with the tokens (x2 here); the 3.88 MB of split-K
 # partials depend only on the item count, which is the same.  None whenever the kernel
 # has changed since that capture.
-DECODE_TRAFFIC_PER_LAUNCH = 2 * 151.23e6 + 3.87e6
+DECODE_TRAFFIC_PER_LAUNCH = 2 * 151.18e6 + 3.88e6
 
 
 def peaks():
