@@ -278,6 +278,7 @@ def run_ours(args, rank, world, dev):
     # prefill write path: 65,536 tokens x 27 layers
     q_stats = bench_quantize(args, dev, world)
     bf16_stats = bench_bf16_baseline(args, dev, world, w, dec_ms)
+    bf16_stats["ours_all_protected"] = bench_all_protected(args, dev, dec_ms)
     cfg_stats = bench_configs(args, dev)
     proj_stats = [bench_projections(args, dev, world, w.batch, w.heads),
                   bench_projections(args, dev, world, W.PAGED_H128.batch, W.PAGED_H128.heads)]
@@ -531,6 +532,40 @@ def bench_bf16_baseline(args, dev, world, w, dec_ms):
             "time_ratio_bf16_over_2bit": round(ms / dec_ms, 3), "capacity_ratio": 4.0}
 
 
+def bench_all_protected(args, dev, dec_ms):
+    """This library's decode with quantization disabled: every token protected (its bf16
+    latent read from the side store, 1,152 B per token with the RoPE key), the same
+    4 x 262,144 tokens at 16 heads as the bench."""
+    w = W.Workload("all_protected_4x256k_h16", 4, (262144,) * 4, 16, n_sink=0, n_recent=262144, seed=1010)
+    try:
+        lay = DecodeLayer(w, 0, dev)
+        lay.fill(w, 0, dev)
+        ws = torch.empty(R.decode_workspace_bytes(w.batch, w.heads), dtype=torch.uint8, device=dev)
+        lens = torch.as_tensor(w.seq_lens, dtype=torch.int32, device=dev)
+        call = lambda: R.decode_attn(lay.cache, lay.params, lay.q_c, lay.q_r, lens, SM_SCALE, lay.out, lay.lse, ws)
+        for _ in range(max(args.warmup, 3)):
+            call()
+        torch.cuda.synchronize()
+        assert R.get_status() == 0
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 10
+        t0.record()
+        for _ in range(reps):
+            call()
+        t1.record()
+        torch.cuda.synchronize()
+        ms = t0.elapsed_time(t1) / reps
+    except Exception as e:                      # report, never lose the bench line
+        return {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+    finally:
+        torch.cuda.empty_cache()
+    nbytes = w.total_tokens * R.BF16_TOKEN_BYTES
+    return {"kernel": "rolaq_decode_split + merge, every token protected (bf16 side store)",
+            "workload": "4 x 262144 tokens, 16 heads, one layer", "bytes_per_token": R.BF16_TOKEN_BYTES,
+            "ms_per_call": round(ms, 4), "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "time_ratio_over_2bit": round(ms / dec_ms, 3)}
+
+
 # ------------------------------------------------------------ profiling cases ----
 # Small single-kernel cases for ncu captures (inputs larger than L2, a few hundred MB on
 # the device): `--case decode` runs one layer of 4 requests x 131,072 tokens at 16 heads,
@@ -538,6 +573,9 @@ def bench_bf16_baseline(args, dev, world, w, dec_ms):
 # output unfold for 32 requests x 128 heads.  They print their own timing.
 
 def run_case(args, dev):
+    if args.case == "protected":
+        print(json.dumps({"case": "protected", "result": bench_all_protected(args, dev, float("nan"))}), flush=True)
+        return
     if args.case == "configs":
         print(json.dumps({"case": "configs", "results": bench_configs(args, dev)}), flush=True)
         return
@@ -657,7 +695,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["decode", "quantize", "project", "configs"], default=None,
+    ap.add_argument("--case", choices=["decode", "quantize", "project", "configs", "protected"], default=None,
                     help="run one small single-kernel case (for ncu captures) instead of the bench")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 1)
