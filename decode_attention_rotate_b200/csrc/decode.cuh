@@ -2,24 +2,27 @@
 // scores (q_c_rot . x + q_R . k_R) * sm_scale with x = mean + scale * level(code),
 // softmax over the request's tokens, 512-d latent readout in the rotated basis.
 //
-// Kernel A (rolaq_decode_split): one CTA per (work item, 16-head chunk).  A work item is a
-// run of whole pages of one request (split-K over the sequence).  Each 64-token page is
-// one tile, handled by warps with fixed roles and handed on through mbarriers:
+// Kernel A (rolaq_decode_split<HC>): one CTA per (work item, chunk of HC = 16 or 32 query
+// heads).  A work item is a run of whole pages of one request (split-K over the sequence),
+// one item per SM in the plan.  Each 64-token page is one tile, handled by warps with
+// fixed roles and handed on through mbarriers:
 //   warp 0 (lane 0)   streams the pages (one 144-row bulk tensor copy each, 128-byte
-//                     swizzle) through kStages shared-memory stages;
+//                     swizzle) through kStages shared-memory stages (3, or 2 with
+//                     32 heads);
 //   warps 8..15       dequantise: thread (token t, group g) forms the four fp16 values
 //                     mean + scale * level of its (token, group) and turns its 128 codes
 //                     into x with one PRMT per pair, stored straight into a 128-byte-
 //                     swizzled x tile [64 tokens][512 channels] (two tiles, double
 //                     buffered).  fp16, not bf16: channels sharing a code share one
 //                     rounding error, which bf16 makes ~5x too large in the output;
-//   warp 1 (lane 0)   issues the tensor-core MMAs: QK as tcgen05.mma M = 64 tokens,
-//                     N = 16 heads, K = 512 (fp16, A = the x tile) plus K = 64 (bf16,
+//   warp 1            issues the tensor-core MMAs (warp-uniform loop, one elected lane
+//                     per batch of instructions): QK as tcgen05.mma M = 64 tokens,
+//                     N = HC heads, K = 512 (fp16, A = the x tile) plus K = 64 (bf16,
 //                     A = the staged page's RoPE rows), S in tensor memory; PV as
-//                     tcgen05.mma M = 128 channels of a group, N = 16 heads, K = 64
+//                     tcgen05.mma M = 128 channels of a group, N = HC heads, K = 64
 //                     tokens, A = the same x tile read transposed (MN-major), B = P,
 //                     O (fp32) accumulated in tensor memory;
-//   warps 4..7        softmax: one tensor-memory load gives a token's 16 scores; the
+//   warps 4..7        softmax: one tensor-memory load gives a token's HC scores; the
 //                     running max moves only when a score exceeds it by more than 2^8
 //                     (a vote in the common case), in which case O is rescaled before
 //                     the next PV; P goes to shared memory as the fp16 B operand.

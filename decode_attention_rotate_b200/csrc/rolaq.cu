@@ -87,7 +87,7 @@ int check_params(const rolaq_layer_params* p) {
     return ROLAQ_OK;
 }
 
-// Split-K target: one work item per SM.  Every 16-head chunk of an item is its own CTA,
+// Split-K target: one work item per SM.  Every head chunk of an item is its own CTA,
 // so with more heads the items run as several waves of equally sized CTAs.
 int decode_target_items() { return current_sms(); }
 
