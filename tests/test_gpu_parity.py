@@ -209,9 +209,20 @@ def test_decode_tiny():
     _decode_case(W.TINY, [256], 16, 0.9816, 1.16)
 
 
-def test_decode_ragged_lengths_and_empty():
-    w = W.Workload("dr", 5, (1, 63, 64, 65, 0), 16, paged_shuffled=True, seed=90)
-    _decode_case(w, [1, 63, 64, 65, 0], 16, 0.9, 1.05)
+@pytest.mark.parametrize("H", [16, 32])
+def test_decode_ragged_lengths_and_empty(H):
+    w = W.Workload("dr", 5, (1, 63, 64, 65, 0), H, paged_shuffled=True, seed=90)
+    _decode_case(w, [1, 63, 64, 65, 0], H, 0.9, 1.05)
+
+
+def test_decode_plan_fits_one_wave():
+    """40 requests of log-uniform lengths: the first chunk size leaves more work items
+    than SMs, so the plan raises it until they fit one wave; every request must still be
+    covered exactly once by its items."""
+    rng = np.random.default_rng(98)
+    lens = [int(x) for x in np.exp(rng.uniform(np.log(64), np.log(20000), size=40)).round()]
+    w = W.Workload("wave", len(lens), tuple(lens), 16, paged_shuffled=True, seed=98)
+    _decode_case(w, lens, 16, 0.92, 1.07)
 
 
 def test_decode_several_splits():
@@ -262,8 +273,9 @@ def test_end_to_end_write_then_decode():
         assert e.max() <= DECODE_TOL, e.max()
 
 
-def test_bad_page_entry_sets_status_and_skips():
-    w = W.Workload("bad", 1, (256,), 16, seed=96)
+@pytest.mark.parametrize("H", [16, 32])
+def test_bad_page_entry_sets_status_and_skips(H):
+    w = W.Workload("bad", 1, (256,), H, seed=96)
     cache, data, _ = build_oracle_cache(w, 0, [256], 0.9, 1.0)
     cache.page_table[0, 1] = cache.num_pages + 5          # outside the pool
     q_c, q_r = W.queries(w, 0)
