@@ -375,7 +375,7 @@ def capture_graph(fn):
 
 
 # ------------------------------------------------------- the other workloads ----
-# Decode on the survey's other decode shapes, each over enough layers that one sweep of
+# Decode on the other decode workloads, each over enough layers that one sweep of
 # the caches exceeds L2 (126 MB): 4 x 32K at 16 heads, 32 requests of log-uniform lengths
 # at 128 heads on shuffled pages, and 64 x 8K with 4 sink + 128 recent bf16 tokens.
 
