@@ -96,6 +96,13 @@ def test_workspace_bytes_shape_rules(lib):
     assert lib.rolaq_decode_workspace_bytes(0, 16) == 0
     n16 = lib.rolaq_decode_workspace_bytes(4, 16)
     assert n16 > 0 and n16 % 16 == 0
+    # (one work item per SM + one per request) x heads x (512 fp32 partial + (m, l))
+    per_item_head = 512 * 4 + 8
+    assert n16 % (16 * per_item_head) == 0
+    sms = n16 // (16 * per_item_head) - 4
+    assert sms >= 1
+    for b, h in [(1, 16), (32, 128), (7, 48), (1000, 32)]:
+        assert lib.rolaq_decode_workspace_bytes(b, h) == (sms + b) * h * per_item_head
 
 
 def test_projection_argument_errors(lib):
