@@ -238,7 +238,7 @@ def run_ours(args, rank, world, dev):
     total_ms = max_over_ranks(total_ms, world)
     ms_per_step = total_ms / args.steps
     step_bytes = cache_bytes_per_step(w)
-    value = step_bytes * world / (ms_per_step * 1e-3) / 1e9
+    value = aggregate_rate(step_bytes, world, ms_per_step)
 
     # end-to-end through the C ABI with host buffers: the step's new tokens and queries come
     # from pinned host memory, the readout goes back to pinned host memory
@@ -273,7 +273,7 @@ def run_ours(args, rank, world, dev):
     e2e_ms = max_over_ranks(t0.elapsed_time(t1), world) / args.steps
     h2d = sum(sum(t.numel() * t.element_size() for t in hi) for hi in host_in)
     d2h = sum(sum(t.numel() * t.element_size() for t in ho) for ho in host_out)
-    e2e_value = step_bytes * world / (e2e_ms * 1e-3) / 1e9
+    e2e_value = aggregate_rate(step_bytes, world, e2e_ms)
 
     # prefill write path: 65,536 tokens x 27 layers
     q_stats = bench_quantize(args, dev, world)
@@ -681,11 +681,19 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The slowest rank's time: every rank passes its own, all get the maximum."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_rate(bytes_per_rank_step, world, ms_per_step):
+    """Whole-job throughput in GB/s: every rank processes its own replica of the workload
+    (weak scaling), timed by the slowest rank."""
+    return bytes_per_rank_step * world / (ms_per_step * 1e-3) / 1e9
 
 
 def main():
