@@ -120,3 +120,20 @@ def test_projection_argument_errors(lib):
     assert uo(o=None) == -1 and uo(v=None) == -1 and uo(b=-1) == -1 and uo(h=0) == -1
     assert uo(w=ptr + 2) == -1
     assert uo(b=0) == 0 and uo(b=0, o=None, v=None) == 0
+
+
+def test_static_decode_rejects_before_any_launch(lib):
+    """The static-scratch decode sizes its plan on the host: shapes it cannot hold fail
+    with ROLAQ_ENOSPACE (and unsupported shapes with their own codes) before any CUDA call."""
+    p = R.rolaq_layer_params(0.9, 1.0, 0.45, 1.5)
+    ptr = 1 << 22
+    def call(batch, heads):
+        c = _cache(batch=max(batch, 1))
+        return lib.rolaq_decode_attn_static(ctypes.byref(c), ctypes.byref(p), ptr, ptr, ptr, batch, heads,
+                                            0.07, ptr, ptr, None)
+    assert call(2, 24) == -4                  # heads not a multiple of 16
+    assert call(2, 0) == -4
+    assert call(0, 16) == -1
+    # 32 MiB / (128 heads x 2,056 B) = 127 items: 127 requests leave no room for a split
+    assert call(127, 128) == -2
+    assert call(5000, 16) == -2               # 1,020 items at 16 heads
