@@ -33,12 +33,15 @@ STATUS_RANGE = 8
 
 
 class RolaqError(RuntimeError):
+    """A C-ABI call returned a negative code; `code` holds it (ROLAQ_E* of rolaq.h)."""
+
     def __init__(self, fn: str, code: int):
         super().__init__(f"{fn} failed: {code} ({strerror(code)})")
         self.code = code
 
 
 class rolaq_cache(ctypes.Structure):
+    """The C descriptor of one layer's paged cache (struct rolaq_cache of rolaq.h)."""
     _fields_ = [
         ("pages_dev", ctypes.c_void_p),
         ("num_pages", ctypes.c_int64),
@@ -52,6 +55,7 @@ class rolaq_cache(ctypes.Structure):
 
 
 class rolaq_layer_params(ctypes.Structure):
+    """Per-layer constants: threshold tau, gain, and the reconstruction levels a, b."""
     _fields_ = [
         ("tau", ctypes.c_float),
         ("gain", ctypes.c_float),
@@ -64,10 +68,12 @@ _LIB = None
 
 
 def library_path() -> str:
+    """Path of the in-tree librolaq.so."""
     return _build.LIB_PATH
 
 
 def lib() -> ctypes.CDLL:
+    """The loaded library with its prototypes; raises when it has not been built."""
     global _LIB
     if _LIB is None:
         path = library_path()
@@ -136,14 +142,17 @@ def _check(fn: str, rc: int) -> None:
 
 
 def version() -> int:
+    """rolaq_version: major * 10000 + minor * 100 + patch."""
     return lib().rolaq_version()
 
 
 def strerror(code: int) -> str:
+    """rolaq_strerror: static description of an error code."""
     return lib().rolaq_strerror(code).decode()
 
 
 def layer_params_init(tau: float, gain: float) -> rolaq_layer_params:
+    """rolaq_layer_params_init: the levels a(tau), b(tau) computed in double, stored fp32."""
     p = rolaq_layer_params()
     _check("rolaq_layer_params_init", lib().rolaq_layer_params_init(ctypes.byref(p), tau, gain))
     return p
@@ -189,6 +198,9 @@ class PagedCache:
 def quantize_append(cache: PagedCache, params: rolaq_layer_params, R_split: torch.Tensor,
                     c: torch.Tensor, k_r: torch.Tensor, req: torch.Tensor, pos: torch.Tensor,
                     seq_lens: Optional[torch.Tensor] = None, stream=None) -> None:
+    """rolaq_quantize_append: write the 2-bit records of n tokens (c bf16 [n, 512], k_r
+    bf16 [n, 64]) at (req[i], pos[i]); seq_lens (request lengths after the append) is
+    needed when the cache has a recent window."""
     n = int(c.shape[0])
     assert c.dtype == torch.bfloat16 and k_r.dtype == torch.bfloat16
     assert req.dtype == torch.int32 and pos.dtype == torch.int32
@@ -199,6 +211,7 @@ def quantize_append(cache: PagedCache, params: rolaq_layer_params, R_split: torc
 
 
 def decode_workspace_bytes(batch: int, heads: int) -> int:
+    """rolaq_decode_workspace_bytes: split-K scratch rolaq_decode_attn needs."""
     return int(lib().rolaq_decode_workspace_bytes(batch, heads))
 
 
@@ -206,6 +219,9 @@ def decode_attn(cache: PagedCache, params: rolaq_layer_params, q_c_rot: torch.Te
                 seq_lens: torch.Tensor, sm_scale: float, out: Optional[torch.Tensor] = None,
                 lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                 stream=None):
+    """rolaq_decode_attn: q_c_rot bf16 [B, H, 512] (rotation folded in), q_r bf16 [B, H, 64]
+    -> (out fp32 [B, H, 512] in the rotated basis, lse fp32 [B, H]); allocates out, lse
+    and the workspace when they are not given."""
     B, H = int(q_c_rot.shape[0]), int(q_c_rot.shape[1])
     assert q_c_rot.dtype == torch.bfloat16 and q_r.dtype == torch.bfloat16
     dev = q_c_rot.device
@@ -288,6 +304,7 @@ def unfold_output(out_rot: torch.Tensor, W_o: torch.Tensor, v: Optional[torch.Te
 
 
 def get_status(stream=None) -> int:
+    """rolaq_get_status: the device status bits (STATUS_*) since the last read; clears them."""
     v = ctypes.c_int(0)
     _check("rolaq_get_status", lib().rolaq_get_status(ctypes.byref(v), _stream(stream)))
     return v.value
