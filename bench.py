@@ -277,11 +277,13 @@ def run_ours(args, rank, world, dev):
 
     # prefill write path: 65,536 tokens x 27 layers
     q_stats = bench_quantize(args, dev, world)
-    bf16_stats = bench_bf16_baseline(args, dev, world, w, dec_ms)
+    # the comparison points and the other workloads are reported beside the headline;
+    # a failure in one of them is recorded in its place instead of losing the line
+    bf16_stats = _guarded(bench_bf16_baseline, args, dev, world, w, dec_ms)
     bf16_stats["ours_all_protected"] = bench_all_protected(args, dev, dec_ms)
-    cfg_stats = bench_configs(args, dev)
-    proj_stats = [bench_projections(args, dev, world, w.batch, w.heads),
-                  bench_projections(args, dev, world, W.PAGED_H128.batch, W.PAGED_H128.heads)]
+    cfg_stats = _guarded(bench_configs, args, dev)
+    proj_stats = [_guarded(bench_projections, args, dev, world, w.batch, w.heads),
+                  _guarded(bench_projections, args, dev, world, W.PAGED_H128.batch, W.PAGED_H128.heads)]
     clocks = sampler.stop()     # sampled across the timed regions
 
     hbm, bf16, src = peaks()
@@ -674,6 +676,13 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------------- plumbing -------
+
+def _guarded(fn, *a):
+    try:
+        return fn(*a)
+    except Exception as e:
+        return {"unavailable": f"{type(e).__name__}: {e}"[:200]}
+
 
 def barrier(world):
     if world > 1:
