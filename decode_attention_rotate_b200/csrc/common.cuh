@@ -17,9 +17,11 @@ __device__ unsigned int g_status;
 
 __device__ __forceinline__ void raise_status(unsigned bits) { atomicOr(&g_status, bits); }
 
-// Spin limit for every mbarrier wait: a wait that exceeds it records
-// ROLAQ_STATUS_TIMEOUT and the waiting thread gives up instead of hanging the GPU.
-constexpr unsigned kSpinLimit = 1u << 24;
+// Every mbarrier wait is bounded: try_wait suspends the thread until the phase completes
+// or a hardware time limit passes, and a wait that has not completed after kWaitCycles
+// SM clocks (about 2 s) records ROLAQ_STATUS_TIMEOUT and gives up instead of hanging
+// the GPU.
+constexpr long long kWaitCycles = 4000000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -54,10 +56,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, unsigned parity) {
 // shared-memory flag of the CTA: the first wait that gives up sets it and every later
 // wait of the CTA returns false at once, so a broken pipeline ends quickly.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity, volatile int* abort) {
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    for (unsigned it = 0; it < kSpinLimit; ++it) {
+    const long long t0 = clock64();
+    for (unsigned it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 1023u) == 1023u && *abort) return false;
+        if ((it & 15u) == 0u) {
+            if (*abort) return false;
+            if (clock64() - t0 > kWaitCycles) break;
+        }
     }
     *abort = 1;
     raise_status(ROLAQ_STATUS_TIMEOUT);
@@ -190,6 +197,12 @@ __device__ __forceinline__ void umma_ss1(uint32_t d, uint64_t da, uint64_t db, u
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
                  :: "r"(d), "l"(da), "l"(db), "r"(idesc), "r"(acc) : "memory");
 }
+// The same with A in tensor memory (`a` = its tensor-memory address).
+__device__ __forceinline__ void umma_ts1(uint32_t d, uint32_t a, uint64_t db, uint32_t idesc, uint32_t acc) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                 :: "r"(d), "r"(a), "l"(db), "r"(idesc), "r"(acc) : "memory");
+}
 // tcgen05.commit from one elected lane of a converged warp.
 __device__ __forceinline__ void umma_commit_warp(uint32_t bar) {
     asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
@@ -215,6 +228,25 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 }
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(addr), "f"(v) : "memory");
+}
+
+// 16 lanes x 256 bits (8 columns): thread i holds lanes i/4 and i/4 + 8 of the 16-lane
+// block at `taddr`, columns 2(i%4) and 2(i%4) + 1 (registers: (lane i/4, column 2(i%4)),
+// (i/4, 2(i%4)+1), (i/4+8, 2(i%4)), (i/4+8, 2(i%4)+1)).
+__device__ __forceinline__ void tmem_st16x256(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1,%2,%3,%4};"
+                 :: "r"(taddr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+// Shared-memory matrix descriptor of an MN-major operand with the 32-byte swizzle: rows of
+// 32 bytes (16 two-byte elements along M or N), 8-row groups `sbo` bytes apart along K.
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr, uint32_t sbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) |
+           (1ull << 46) | (6ull << 61);
 }
 
 // 128-byte swizzle of a (row, byte) position inside a 1024-byte aligned tile:

@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_tm.cuh"
 #include "project.cuh"
 #include "quantize.cuh"
 
@@ -15,6 +16,9 @@ using namespace rolaq;
 namespace {
 
 constexpr int kVersion = 100;   // 0.1.0
+// The tensor-memory-operand decode (decode_tm.cuh) takes 16-head chunks once it beats the
+// shared-memory decode on the long-context workload; until then both are built.
+constexpr bool kDecodeTm = false;
 constexpr int kMaxDevices = 64;
 
 int device_sms(int dev) {
@@ -148,6 +152,19 @@ int rolaq_layer_params_init(rolaq_layer_params* p, float tau, float gain) {
     return ROLAQ_OK;
 }
 
+int rolaq_coupled_gain(float tau, double* gain, double* kappa1) {
+    if (!gain || !isfinite(tau) || !(tau > 0.f)) return ROLAQ_EINVAL;
+    const double t = tau;
+    const double inv_sqrt_2pi = 0.39894228040143267794;
+    const double phi0 = inv_sqrt_2pi, phit = inv_sqrt_2pi * exp(-0.5 * t * t);
+    const double a = (phi0 - phit) / (0.5 * erf(t / sqrt(2.0)));
+    const double b = phit / (0.5 * erfc(t / sqrt(2.0)));
+    const double k1 = 2.0 * (a * (phi0 - phit) + b * phit);
+    *gain = 1.0 / k1;
+    if (kappa1) *kappa1 = k1;
+    return ROLAQ_OK;
+}
+
 int rolaq_prepare_rotation(const float* R_dev, void* R_split_dev, void* stream) {
     if (!R_dev || !R_split_dev || !aligned(R_dev, 4) || !aligned(R_split_dev, 16)) return ROLAQ_EINVAL;
     rolaq_split_rotation<<<ROLAQ_D_C, 128, 0, (cudaStream_t)stream>>>(
@@ -231,6 +248,23 @@ size_t rolaq_decode_workspace_bytes(int batch, int heads) {
     return decode_ws_bytes(batch, heads);
 }
 
+// Argument checks shared by both decode entry points (everything but the workspace).
+static int decode_check(const rolaq_cache* cache, const rolaq_layer_params* p, const void* q_c_rot_dev,
+                        const void* q_R_dev, const int32_t* seq_lens_dev, int batch, int heads,
+                        float sm_scale, const float* out_dev, const float* lse_dev) {
+    int rc = check_cache(cache);
+    if (rc) return rc;
+    if ((rc = check_params(p))) return rc;
+    if (heads <= 0 || heads % 16) return ROLAQ_EUNSUPPORTED;
+    if (batch <= 0 || batch > cache->batch) return ROLAQ_EINVAL;
+    if (!q_c_rot_dev || !q_R_dev || !seq_lens_dev || !out_dev) return ROLAQ_EINVAL;
+    if (!aligned(q_c_rot_dev, 4) || !aligned(q_R_dev, 4) || !aligned(seq_lens_dev, 4) ||
+        !aligned(out_dev, 16) || (lse_dev && !aligned(lse_dev, 4)))
+        return ROLAQ_EINVAL;
+    if (!isfinite(sm_scale)) return ROLAQ_EINVAL;
+    return ROLAQ_OK;
+}
+
 // The decode with an explicit split-K target (work items before the per-request
 // remainders); the workspace must hold (target + batch) items.
 static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* p,
@@ -238,16 +272,9 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
                             const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
                             float* out_dev, float* lse_dev,
                             void* workspace_dev, size_t workspace_bytes, void* stream, int target) {
-    int rc = check_cache(cache);
+    int rc = decode_check(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale, out_dev, lse_dev);
     if (rc) return rc;
-    if ((rc = check_params(p))) return rc;
-    if (heads <= 0 || heads % 16) return ROLAQ_EUNSUPPORTED;
-    if (batch <= 0 || batch > cache->batch) return ROLAQ_EINVAL;
-    if (!q_c_rot_dev || !q_R_dev || !seq_lens_dev || !out_dev || !workspace_dev) return ROLAQ_EINVAL;
-    if (!aligned(q_c_rot_dev, 4) || !aligned(q_R_dev, 4) || !aligned(seq_lens_dev, 4) ||
-        !aligned(out_dev, 16) || !aligned(workspace_dev, 16) || (lse_dev && !aligned(lse_dev, 4)))
-        return ROLAQ_EINVAL;
-    if (!isfinite(sm_scale)) return ROLAQ_EINVAL;
+    if (!workspace_dev || !aligned(workspace_dev, 16)) return ROLAQ_EINVAL;
     if (target < 1) return ROLAQ_ENOSPACE;
     if (workspace_bytes < decode_ws_bytes_for(batch, heads, target)) return ROLAQ_ENOSPACE;
 
@@ -279,10 +306,22 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
     a.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace_dev) +
                                         (size_t)items_cap * heads * ROLAQ_D_C * sizeof(float));
 
-    // 32 heads per CTA when the head count allows it (twice the work per tensor-core
-    // instruction and per dequantised tile), else 16
     cudaStream_t s = (cudaStream_t)stream;
-    if (heads % 32 == 0) {
+    if (heads % 32 != 0 && kDecodeTm) {
+        // 16 heads per CTA, both tensor-core A operands in tensor memory
+        CUtensorMap map_cm, map_kr;
+        if (!encode_2d(&map_cm, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache->pages_dev, 128, rows, 128, 128, kTmCmRows,
+                       CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_2d(&map_kr, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache->pages_dev, 128, rows, 128, 128, kTmKrRows,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+            return ROLAQ_ECUDA;
+        const size_t smem = sizeof(TmSmem) + 1024;
+        static bool attr_done[kMaxDevices] = {false};
+        set_smem_limit_once(rolaq_decode_tm, smem, attr_done);
+        rolaq_decode_tm<<<dim3(items_cap, heads / kTmHeads), kTmThreads, smem, s>>>(map_cm, map_kr, a);
+    } else if (heads % 32 == 0) {
+        // 32 heads per CTA (twice the work per tensor-core instruction and per
+        // dequantised tile)
         const size_t smem = sizeof(DecodeSmem<32>) + 1024;
         static bool attr_done[kMaxDevices] = {false};
         set_smem_limit_once(rolaq_decode_split<32>, smem, attr_done);
@@ -337,8 +376,8 @@ int rolaq_decode_attn_static(const rolaq_cache* cache, const rolaq_layer_params*
                              const void* q_c_rot_dev, const void* q_R_dev,
                              const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
                              float* out_dev, float* lse_dev, void* stream) {
-    if (heads <= 0 || heads % 16) return ROLAQ_EUNSUPPORTED;
-    if (batch <= 0) return ROLAQ_EINVAL;
+    int rc = decode_check(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale, out_dev, lse_dev);
+    if (rc) return rc;
     // as many split-K items as the fixed array holds, up to one per SM
     const long long fit = (long long)(ROLAQ_STATIC_SCRATCH_BYTES / decode_item_bytes(heads)) - batch;
     const int target = (int)(fit < decode_target_items() ? fit : decode_target_items());

@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.rolaq_version.restype = i32
         L.rolaq_strerror.restype = ctypes.c_char_p
         L.rolaq_strerror.argtypes = [i32]
+        L.rolaq_coupled_gain.restype = i32
+        L.rolaq_coupled_gain.argtypes = [ctypes.c_float, P(ctypes.c_double), P(ctypes.c_double)]
         L.rolaq_layer_params_init.restype = i32
         L.rolaq_layer_params_init.argtypes = [P(rolaq_layer_params), ctypes.c_float, ctypes.c_float]
         L.rolaq_prepare_rotation.restype = i32
@@ -149,6 +151,13 @@ def version() -> int:
 def strerror(code: int) -> str:
     """rolaq_strerror: static description of an error code."""
     return lib().rolaq_strerror(code).decode()
+
+
+def coupled_gain(tau: float):
+    """rolaq_coupled_gain: (gain giving unit response at threshold tau, E[z level(z)])."""
+    g, k = ctypes.c_double(), ctypes.c_double()
+    _check("rolaq_coupled_gain", lib().rolaq_coupled_gain(tau, ctypes.byref(g), ctypes.byref(k)))
+    return g.value, k.value
 
 
 def layer_params_init(tau: float, gain: float) -> rolaq_layer_params:
@@ -250,11 +259,15 @@ def decode_attn_static(cache: PagedCache, params: rolaq_layer_params, q_c_rot: t
     that cannot allocate device memory.  out / lse must be passed by such callers (the
     defaults here allocate them for convenience)."""
     B, H = int(q_c_rot.shape[0]), int(q_c_rot.shape[1])
+    assert q_c_rot.dtype == torch.bfloat16 and q_r.dtype == torch.bfloat16
+    assert tuple(q_c_rot.shape) == (B, H, D_C) and tuple(q_r.shape) == (B, H, D_R)
     dev = q_c_rot.device
     if out is None:
         out = torch.empty((B, H, D_C), dtype=torch.float32, device=dev)
     if lse is None:
         lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    assert out.dtype == torch.float32 and out.is_contiguous() and tuple(out.shape) == (B, H, D_C)
+    assert lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H)
     d = cache.desc()
     _check("rolaq_decode_attn_static", lib().rolaq_decode_attn_static(
         ctypes.byref(d), ctypes.byref(params), _ptr(q_c_rot), _ptr(q_r), _ptr(seq_lens), B, H,

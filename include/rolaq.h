@@ -11,6 +11,8 @@
  *           reconstruction around the group mean.
  *   [S3.3]  §3.3 "Joint Calibration and Inference": serving stores rotated latents as
  *           2-bit codes and folds the read-side rotation into the absorbed projections.
+ *   [B.3]   §B.3: at the official threshold the MSE-optimal response is about 0.88;
+ *           the coupled gain restores unit response.
  *   [S4.1]  §4.1 "Setup": protection keeps the first 4 sink and the most recent tokens
  *           in BF16.
  *   [A.3]   §A.3 "Calibration and Storage": 288 B per unprotected token per layer
@@ -128,6 +130,17 @@ typedef struct rolaq_layer_params {
  * tau or gain.  [S3.2]                                                                */
 int rolaq_layer_params_init(rolaq_layer_params* p, float tau, float gain);
 
+/* Coupled gain for threshold tau > 0 [S3.2], [B.3]: the gain links to the threshold so
+ * that the centered reconstruction has unit response.  With z ~ N(0, 1) and the centroid
+ * levels of tau, the response of the reconstruction gain * level(z) is
+ *   kappa(tau) = gain * E[z * level(z)] = gain * 2 (a (phi(0) - phi(tau)) + b phi(tau)),
+ * so the coupled gain is 1 / E[z * level(z)].  Computed on the host in double.  Writes the
+ * coupled gain to *gain and, when kappa1 is not NULL, E[z * level(z)] (the response at
+ * gain 1; about 0.8825 at the Lloyd-Max threshold 0.9816, where the coupled gain is
+ * about 1.1331) to *kappa1.  Returns ROLAQ_EINVAL for a NULL gain or a non-finite or
+ * non-positive tau.  Pass the result to rolaq_layer_params_init as the layer's gain.      */
+int rolaq_coupled_gain(float tau, double* gain, double* kappa1);
+
 /* Convert the fp32 rotation R_dev [512][512] (row-major, y = c . R for a row vector c)
  * into the tensor-core operand R_split_dev (ROLAQ_RSPLIT_BYTES, 16-B aligned): plane 0
  * holds bf16(R^T), plane 1 the nearest bf16 of R^T - plane0, plane 2 the nearest bf16 of
@@ -187,6 +200,13 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
  * cudaMalloc: code running while a memory pool or a captured allocator owns the device
  * memory, plug-ins that are handed tensors but no allocator, and hosts that forbid
  * allocation after start-up.  The call itself allocates nothing.
+ *   - The array is part of the library's device code, so the 32 MiB are committed on a
+ *     device when the library's module is loaded there: at the first call of any librolaq
+ *     entry point that reaches that device (with lazy module loading), not only at the
+ *     first call of this one.  Every process that loads the library pays it on each device
+ *     it uses, whether or not it calls this entry point.  ROLAQ_ECUDA from the first call
+ *     on a device can mean that this load failed (for instance because a memory pool
+ *     already holds nearly all of the device's memory).
  *   - The first call on each device looks up the array's device address on that device;
  *     make that first call before any stream capture.
  *   - The split-K plan uses as many work items as the array holds, up to one per SM:

@@ -283,11 +283,9 @@ def pages_read_fast(pool: np.ndarray, page_table: np.ndarray, req: int, L: int):
 
 
 def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bfloat16 bit patterns (uint16) as fp64 values: a bfloat16 is the upper half of an
+    IEEE fp32, so the pattern moves into bits 16..31 of a 32-bit word read as fp32."""
     return (np.asarray(bits, np.uint32) << 16).astype(np.uint32).view(np.float32).astype(np.float64)
-
-
-def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    return (np.ascontiguousarray(bf16_round(x).astype(np.float32)).view(np.uint32) >> 16).astype(np.uint16)
 
 
 # ---- absorbed projections around the cache (RoLaQ §3.3; Fig. 3a) -----------------

@@ -4,6 +4,7 @@ import ctypes
 import math
 import subprocess
 
+import numpy as np
 import pytest
 
 from decode_attention_rotate_b200 import build as B
@@ -58,6 +59,22 @@ def _cache(**kw):
     c.n_sink = kw.get("n_sink", 0)
     c.n_recent = kw.get("n_recent", 0)
     return c
+
+
+def test_coupled_gain_matches_oracle(lib):
+    """rolaq_coupled_gain against the oracle's coupled gain over the learned threshold
+    range 0.85-1.1 (RoLaQ §C.3) and at the Lloyd-Max threshold (gain 1.1331, response at
+    gain 1 about 0.88, §B.3); invalid thresholds are refused."""
+    for tau in np.linspace(0.85, 1.1, 11):
+        tau32 = float(np.float32(tau))
+        g, k = R.coupled_gain(tau32)
+        assert abs(g - O.coupled_gain(tau32)) < 1e-12
+        assert abs(k - O.response(tau32, 1.0)) < 1e-12
+    g, k = R.coupled_gain(0.9816)
+    assert abs(g - 1.1331) < 1e-4 and abs(k - 0.8825) < 1e-4
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        with pytest.raises(R.RolaqError):
+            R.coupled_gain(bad)
 
 
 def test_decode_argument_errors(lib):
@@ -137,3 +154,13 @@ def test_static_decode_rejects_before_any_launch(lib):
     # 32 MiB / (128 heads x 2,056 B) = 127 items: 127 requests leave no room for a split
     assert call(127, 128) == -2
     assert call(5000, 16) == -2               # 1,020 items at 16 heads
+    # the shared argument checks come first: a batch beyond the cache, a null cache or a
+    # null output give ROLAQ_EINVAL even where the scratch could not hold the plan
+    c = _cache(batch=4)
+    assert lib.rolaq_decode_attn_static(ctypes.byref(c), ctypes.byref(p), ptr, ptr, ptr, 5000, 16,
+                                        0.07, ptr, ptr, None) == -1
+    assert lib.rolaq_decode_attn_static(None, ctypes.byref(p), ptr, ptr, ptr, 5000, 16,
+                                        0.07, ptr, ptr, None) == -1
+    c = _cache(batch=5000)
+    assert lib.rolaq_decode_attn_static(ctypes.byref(c), ctypes.byref(p), ptr, ptr, ptr, 5000, 16,
+                                        0.07, None, ptr, None) == -1

@@ -92,6 +92,61 @@ def test_response_by_monte_carlo():
     assert abs((z * ell).mean() - O.response(tau, 1.0)) < 3e-3
 
 
+def test_stored_scale_is_gain_times_population_std():
+    """Metadata is (mean, gain * population std) per group (RoLaQ §3.2: the gain scales the
+    reconstruction around the group mean).  Closed forms with R = I: an arithmetic
+    progression 0..127 has mean 63.5 and population std sqrt((128^2 - 1) / 12); an
+    alternating +-1 group has mean 0 and std 1."""
+    gain = 1.16
+    c = np.zeros((1, 512))
+    c[0, :128] = np.arange(128.0)
+    c[0, 128:256] = np.where(np.arange(128) % 2 == 0, 1.0, -1.0)
+    c[0, 256:384] = 3.0 * np.arange(128.0) - 7.0
+    c[0, 384:] = np.where(np.arange(128) % 2 == 0, 0.25, -0.25)
+    q = O.quantize(c, np.eye(512), 0.9816, gain)
+    sd_ap = math.sqrt((128 ** 2 - 1) / 12.0)
+    expect = [(63.5, gain * sd_ap), (0.0, gain), (3.0 * 63.5 - 7.0, gain * 3.0 * sd_ap), (0.0, gain * 0.25)]
+    for gi, (mu, sc) in enumerate(expect):
+        assert q["meta"][0, gi, 0] == np.float32(mu)
+        assert q["meta"][0, gi, 1] == np.float32(sc)
+
+
+def test_reconstruction_response_scales_with_gain():
+    """For Gaussian latents the centered reconstruction (x - mean) / std has response
+    E[z (x - mean) / std] = g * kappa(tau) (RoLaQ §3.2, §B.3): at tau = 0.9816 and g = 1.16,
+    1.16 * 0.8825.  kappa by quadrature; Monte Carlo over 2,048,000 coordinates standardised
+    within their 128-groups (the within-group standardisation moves the mean by well under
+    the 1e-2 tolerance)."""
+    tau, gain = 0.9816, 1.16
+    rng = np.random.default_rng(11)
+    c = rng.standard_normal((4000, 512))
+    q = O.quantize(c, np.eye(512), tau, gain)
+    x = O.dequantize(q["packed"], q["meta"], tau)
+    y = q["y"].reshape(-1, 4, 128)
+    mu, sd = q["mu"][:, :, None], q["sd"][:, :, None]
+    z = (y - mu) / sd
+    resp = (z * (x.reshape(-1, 4, 128) - mu) / sd).mean()
+    qa, qb = centroids_by_quadrature(tau)
+    pdf = stats.norm.pdf
+    kappa = 2 * (qa * integrate.quad(lambda v: v * pdf(v), 0, tau)[0]
+                 + qb * integrate.quad(lambda v: v * pdf(v), tau, np.inf)[0])
+    assert abs(resp - gain * kappa) < 1e-2
+
+
+def test_bf16_bits_decode_matches_torch():
+    """bfloat16 bit patterns decode like torch's bfloat16 view (all non-NaN patterns of a
+    random sample plus hand values: 0x3F80 = 1, 0xC000 = -2, 0x0001 = 2^-133, 0x7F7F the
+    largest finite)."""
+    rng = np.random.default_rng(12)
+    bits = rng.integers(0, 1 << 16, 20000).astype(np.uint16)
+    bits = bits[~(((bits & 0x7F80) == 0x7F80) & ((bits & 0x007F) != 0))]
+    ref = torch.as_tensor(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    got = O.bf16_bits_to_f64(bits)
+    assert (got == ref).all()
+    hand = O.bf16_bits_to_f64(np.array([0x3F80, 0xC000, 0x0001, 0x7F7F], np.uint16))
+    assert list(hand) == [1.0, -2.0, 2.0 ** -133, (2 - 2 ** -7) * 2.0 ** 127]
+
+
 # ------------------------------------------------------------- storage ----------
 
 def test_storage_accounting_matches_pages():
@@ -394,6 +449,24 @@ def test_planted_mistakes_are_caught(monkeypatch):
             assert _pins_fail(m, name, bad, pins) == len(pins), name
     assert O.levels is good_levels and O.group_stats is good_stats
     assert O.pack is good_pack and O.assign is good_assign
+
+
+def test_planted_gain_mistakes_are_caught(monkeypatch):
+    """Dropping the gain from the stored scale, or applying it twice, fails both scale pins."""
+    good = O.quantize
+    pins = [test_stored_scale_is_gain_times_population_std, test_reconstruction_response_scales_with_gain]
+    for bad in (lambda c, R, tau, gain: good(c, R, tau, 1.0),
+                lambda c, R, tau, gain: good(c, R, tau, gain * gain)):
+        with monkeypatch.context() as m:
+            assert _pins_fail(m, "quantize", bad, pins) == len(pins)
+    assert O.quantize is good
+
+
+def test_planted_bf16_decode_mistake_is_caught(monkeypatch):
+    """A wrong shift in the bfloat16 bit decode fails its pin."""
+    bad = lambda bits: (np.asarray(bits, np.uint32) << 15).astype(np.uint32).view(np.float32).astype(np.float64)
+    with monkeypatch.context() as m:
+        assert _pins_fail(m, "bf16_bits_to_f64", bad, [test_bf16_bits_decode_matches_torch]) == 1
 
 
 def test_planted_transposed_rotation_is_caught(monkeypatch):
