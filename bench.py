@@ -33,12 +33,30 @@ METRIC = "2-bit MLA decode: cache GB/s & % HBM roofline; quantize-append tokens/
 SM_SCALE = 1.0 / math.sqrt(192.0)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-# DRAM bytes (read + write) of the split kernel per decode launch of the bench workload,
-# from the ncu capture summarised in profiles/decode_split_4x128k_h16.md (4 x 131,072
-# tokens): the 151.18 MB of reads scale with the tokens (x2 here); the 3.88 MB of split-K
-# partials depend only on the item count, which is the same.  None whenever the kernel
-# has changed since that capture.
-DECODE_TRAFFIC_PER_LAUNCH = 2 * 151.18e6 + 3.88e6
+# DRAM bytes (read + write) of the decode kernel per launch of the bench workload, taken
+# from one ncu capture of the 4 x 131,072-token case (dram__bytes_read.sum +
+# dram__bytes_write.sum; the reads scale with the tokens, x2 here, the split-K partials
+# depend only on the item count, which is the same), together with the SHA-256 of the
+# decode kernel sources it was taken on.  The bench reports it only while those sources
+# are unchanged, and null otherwise.
+DECODE_TRAFFIC = {"sources_sha256": None, "bytes_per_launch": None}
+DECODE_SOURCES = ("common.cuh", "decode.cuh", "decode_tm.cuh")
+
+
+def decode_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "decode_attention_rotate_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def decode_traffic():
+    """Measured DRAM bytes per decode launch, or None once the kernel sources changed."""
+    if DECODE_TRAFFIC["sources_sha256"] and DECODE_TRAFFIC["sources_sha256"] == decode_sources_sha256():
+        return DECODE_TRAFFIC["bytes_per_launch"]
+    return None
 
 
 def peaks():
@@ -299,7 +317,7 @@ def run_ours(args, rank, world, dev):
                    "l2": "inputs larger than L2 (8.15 GB cache per step), no flush",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": DECODE_TRAFFIC_PER_LAUNCH,
+                     "frac": round(achieved / hbm, 4), "traffic": decode_traffic(),
                      "kernel": "decode call (split + merge launches); traffic: split kernel",
                      "peak_source": src,
                      "bytes_per_launch": dec_bytes, "ms_per_launch": round(dec_ms, 4),

@@ -40,6 +40,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
 }
+// Arrive from lane 0 of the warp only (a predicated instruction, no branch).
+__device__ __forceinline__ void mbar_arrive_lane0(uint32_t bar) {
+    asm volatile("{\n\t.reg .pred p;\n\t.reg .u32 l;\n\tmov.u32 l, %%laneid;\n\t"
+                 "setp.eq.u32 p, l, 0;\n\t@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}"
+                 :: "r"(bar) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, unsigned bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
                  :: "r"(bar), "r"(bytes) : "memory");
@@ -52,6 +58,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, unsigned parity) {
                  : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
+// Up to 64 polls of try_wait in one PTX loop (three instructions per poll, no
+// compiler-inserted yields); true once the phase has completed.
+__device__ __forceinline__ bool mbar_poll64(uint32_t bar, unsigned parity) {
+    unsigned ok;
+    asm volatile("{\n\t.reg .pred p, q;\n\t.reg .u32 n;\n\t"
+                 "mov.u32 n, 0;\n"
+                 "ROLAQ_POLL_%=:\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "@p bra ROLAQ_POLL_DONE_%=;\n\t"
+                 "add.u32 n, n, 1;\n\t"
+                 "setp.lt.u32 q, n, 64;\n\t"
+                 "@q bra ROLAQ_POLL_%=;\n"
+                 "ROLAQ_POLL_DONE_%=:\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
 // Bounded wait; false (and a status bit) when the phase never completes.  `abort` is a
 // shared-memory flag of the CTA: the first wait that gives up sets it and every later
 // wait of the CTA returns false at once, so a broken pipeline ends quickly.
@@ -59,16 +82,37 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     const long long t0 = clock64();
-    for (unsigned it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 15u) == 0u) {
-            if (*abort) return false;
-            if (clock64() - t0 > kWaitCycles) break;
-        }
+    for (;;) {
+        if (mbar_poll64(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > kWaitCycles) break;
     }
     *abort = 1;
     raise_status(ROLAQ_STATUS_TIMEOUT);
     return false;
+}
+
+// Bounded wait for whichever of two barriers completes its phase first: 0 or 1, or -1
+// when the CTA aborts or the wait gives up.  Called by a whole warp; lane 0 decides.
+__device__ __forceinline__ int mbar_wait_either(uint32_t bar0, uint32_t bar1, unsigned parity,
+                                                volatile int* abort) {
+    int which = -1;
+    if ((threadIdx.x & 31) == 0) {
+        const long long t0 = clock64();
+        for (unsigned it = 0;; ++it) {
+            if (mbar_try_wait(bar0, parity)) { which = 0; break; }
+            if (mbar_try_wait(bar1, parity)) { which = 1; break; }
+            if ((it & 15u) == 15u) {
+                if (*abort) break;
+                if (clock64() - t0 > kWaitCycles) {
+                    *abort = 1;
+                    raise_status(ROLAQ_STATUS_TIMEOUT);
+                    break;
+                }
+            }
+        }
+    }
+    return __shfl_sync(0xffffffffu, which, 0);
 }
 
 // ------------------------------------------------------- bulk tensor copies -----
@@ -150,6 +194,29 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// 32 lanes x 8 columns of 32-bit words, one lane per thread.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&u)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&u)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 :: "r"(taddr), "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]),
+                    "r"(u[7])
+                 : "memory");
+}
+// 16 lanes x 16 columns, twice: threads 0-15 write lanes 0-15 of the quarter at `taddr`,
+// threads 16-31 the same lanes 64 columns further.
+__device__ __forceinline__ void tmem_st16x32bx2_64(uint32_t taddr, const uint32_t (&u)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 64, "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        :: "r"(taddr), "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]),
+           "r"(u[7]), "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]),
+           "r"(u[14]), "r"(u[15])
+        : "memory");
 }
 // 32 lanes x 16 columns of 32-bit words, one lane per thread.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&u)[16]) {

@@ -45,7 +45,8 @@ constexpr int kMetaRow = 64;                        // page rows: codes 0..63, m
 constexpr int kKrRow = 80;                          // RoPE keys 80..143
 constexpr int kSCol = 0;                            // TMEM: S tiles at columns 0 and HC
 constexpr int kOCol = 64;                           //       O at 64.. (HC per group)
-template <int HC> __host__ __device__ constexpr int tmem_cols_for() { return HC == 16 ? 128 : 256; }
+constexpr int kXqCol = 256;                         //       token-major x (QK's A): 256..511
+template <int HC> __host__ __device__ constexpr int tmem_cols_for() { return 512; }
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kF16Max = 65504.f;
 
@@ -82,6 +83,8 @@ struct DecodeSmem {
     alignas(8) uint64_t pfree[kStages];    // page read by the dequant warps and the QK MMAs
     alignas(8) uint64_t xready[2][2];      // x tile half written (channel groups 0-1 / 2-3)
     alignas(8) uint64_t xfree[2][2];       // PV of the tile done for groups 0-1 / all groups
+    alignas(8) uint64_t xq_full[2];        // token-major x in tensor memory written (groups 0-1 / 2-3)
+    alignas(8) uint64_t xq_free;           // QK of the page done with the token-major x
     alignas(8) uint64_t sfull[2];          // QK of the tile done
     alignas(8) uint64_t sfree[2];          // scores read by the softmax warps
     alignas(8) uint64_t pready[2];         // P written (and O rescaled if needed)
@@ -370,6 +373,8 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             mbar_init(smem_u32(&sm.sfree[s]), 4);
             mbar_init(smem_u32(&sm.pready[s]), 4);
         }
+        for (int hf = 0; hf < 2; ++hf) mbar_init(smem_u32(&sm.xq_full[hf]), (kDecodeThreads / 32 - kDqWarp0) / 2);
+        mbar_init(smem_u32(&sm.xq_free), 1);
         for (int h = 0; h < HC; ++h) sm.mref[h] = -INFINITY;
         sm.abort = 0;
         fence_mbar_init();
@@ -460,18 +465,21 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                 const uint64_t da = dxk + (uint64_t)(bi * (kXTile >> 4));
                 const uint64_t dk = dkr + (uint64_t)(st * (ROLAQ_PAGE_BYTES >> 4));
                 const uint32_t d = tmem + kSCol + HC * bi;
-                // channel groups 0-1 (K steps 0..15) as soon as that half of the tile is written
+                // QK from the token-major x in tensor memory (M = 64: token r in lane
+                // 32 (r / 16) + r % 16), channel groups 0-1 (K steps 0..15) as soon as that
+                // half is written, then groups 2-3 and the RoPE keys
+                (void)da;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    mbar_wait(smem_u32(&sm.xready[bi][hf]), (unsigned)((i >> 1) & 1), &sm.abort);
+                    mbar_wait(smem_u32(&sm.xq_full[hf]), (unsigned)(i & 1), &sm.abort);
                     __syncwarp();
                     tc_fence_after();
                     if (elect_one()) {
 #pragma unroll
                         for (int k2 = 0; k2 < ROLAQ_D_C / 32; ++k2) {
                             const int kk = hf * (ROLAQ_D_C / 32) + k2;
-                            umma_ss1(d, da + (uint64_t)(((kk >> 2) * kXAtom + (kk & 3) * 32) >> 4),
-                                     dqc + (uint64_t)((kk * 256) >> 4), kIdQk, kk > 0 ? 1u : 0u);
+                            umma_ts1(d, tmem + kXqCol + 8 * kk, dqc + (uint64_t)((kk * 256) >> 4), kIdQk,
+                                     kk > 0 ? 1u : 0u);
                         }
                         if (hf == 1) {
 #pragma unroll
@@ -480,6 +488,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                                          kIdRope, 1u);
                             umma_commit(smem_u32(&sm.sfull[bi]));
                             umma_commit(smem_u32(&sm.pfree[st]));
+                            umma_commit(smem_u32(&sm.xq_free));
                         }
                     }
                     __syncwarp();
@@ -493,6 +502,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
         // warps 8..11 take channel groups 0-1, warps 12..15 groups 2-3
         const int wq = warp - kDqWarp0, hf = wq >> 2;
         const int t = 16 * (wq & 3) + (lane & 15), g = 2 * hf + (lane >> 4);
+        const uint32_t xq_lane = (uint32_t)(32 * (warp & 3)) << 16;      // this warp's lane quarter
         const bool protect = args.n_sink > 0 || args.n_recent > 0;
         const int nslot = args.n_sink + args.n_recent;
         const float la = args.level_a, lb = args.level_b;
@@ -511,6 +521,23 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             dequant_tile_part(sm.stage[st], t, g, valid, prot, prow, la, lb, o);
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.pfree[st]));      // this warp is done with the page
+            // token-major x for QK: lanes 0-15 of this warp's quarter are the tokens, threads
+            // 0-15 write group 2 hf and threads 16-31 group 2 hf + 1 (64 columns further)
+            if (i >= 1) mbar_wait(smem_u32(&sm.xq_free), (unsigned)((i - 1) & 1), &sm.abort);
+            __syncwarp();
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[16];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) { v[j] = o[2 * c][j]; v[8 + j] = o[2 * c + 1][j]; }
+                tmem_st16x32bx2_64(tmem + xq_lane + kXqCol + 128 * hf + 16 * c, v);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&sm.xq_full[hf]));
+            // the shared-memory copy (PV's A operand, read MN-major)
             if (i >= 2) mbar_wait(smem_u32(&sm.xfree[bi][hf]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
             store_tile_part(sm.x[bi], t, g, o);
             fence_proxy_async_smem();

@@ -69,13 +69,13 @@ struct TmSmem {
     alignas(128) uint8_t qr[kTmHeads * ROLAQ_D_R * 2];          // bf16 RoPE query
     alignas(1024) uint8_t P[2][kTmTok * 32];                    // fp16 probabilities, PV B
     uint4 tbl[3][ROLAQ_GROUPS][kTmTok / 4];                     // fp16x2 (sc01, sc23, mu01, mu23)
-    float red[4][kTmHeads];
+    float red[2][4][kTmHeads / 2];
     float mref[kTmHeads];
     float alpha[kTmHeads];
-    int vote[2][4];
+    int vote[2][2][4];
     alignas(8) uint64_t full[kTmStages];
     uint64_t pfree[kTmStages];
-    uint64_t xq_full, xq_free;
+    uint64_t xq_full[2], xq_free[2];       // token-major x, channel groups 0-1 / 2-3
     uint64_t tbl_full[3], tbl_free[3];
     uint64_t xp_full[kTmXpSlots], xp_free[kTmXpSlots];
     uint64_t sfull[2], sfree[2], pready[2], pvdone[2];
@@ -186,20 +186,22 @@ rolaq_decode_tm(const __grid_constant__ CUtensorMap map_cm, const __grid_constan
             mbar_init(smem_u32(&sm.full[s]), 1);
             mbar_init(smem_u32(&sm.pfree[s]), 8 + 8 + 1);      // expansion warps + RoPE MMAs
         }
-        mbar_init(smem_u32(&sm.xq_full), 8);
+        for (int hx = 0; hx < 2; ++hx) {
+            mbar_init(smem_u32(&sm.xq_full[hx]), 4);
+            mbar_init(smem_u32(&sm.xq_free[hx]), 1);
+        }
         for (int k3 = 0; k3 < 3; ++k3) {
             mbar_init(smem_u32(&sm.tbl_full[k3]), 8);
             mbar_init(smem_u32(&sm.tbl_free[k3]), 8);
         }
-        mbar_init(smem_u32(&sm.xq_free), 1);
         for (int sl = 0; sl < kTmXpSlots; ++sl) {
             mbar_init(smem_u32(&sm.xp_full[sl]), 4);
             mbar_init(smem_u32(&sm.xp_free[sl]), 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_u32(&sm.sfull[s]), 1);
-            mbar_init(smem_u32(&sm.sfree[s]), 4);
-            mbar_init(smem_u32(&sm.pready[s]), 4);
+            mbar_init(smem_u32(&sm.sfree[s]), 8);
+            mbar_init(smem_u32(&sm.pready[s]), 8);
             mbar_init(smem_u32(&sm.pvdone[s]), 1);
         }
         for (int h = 0; h < kTmHeads; ++h) sm.mref[h] = -INFINITY;
@@ -281,23 +283,38 @@ rolaq_decode_tm(const __grid_constant__ CUtensorMap map_cm, const __grid_constan
         for (int i = 0; i < nt; ++i) {
             {
                 const int bi = i & 1, st = i % kTmStages;
-                mbar_wait(smem_u32(&sm.xq_full), (unsigned)(i & 1), &sm.abort);
-                mbar_wait(smem_u32(&sm.full[st]), (unsigned)((i / kTmStages) & 1), &sm.abort);
+                const uint32_t d = tmem + kTmColS + kTmHeads * bi;
                 if (i >= 2) mbar_wait(smem_u32(&sm.sfree[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
+                // the two halves of x (channel groups 0-1, 2-3) in the order they are
+                // written; the first initialises S, the second adds the RoPE keys
+                const int first = mbar_wait_either(smem_u32(&sm.xq_full[0]), smem_u32(&sm.xq_full[1]),
+                                                   (unsigned)(i & 1), &sm.abort);
+                const int hf0 = first < 0 ? 0 : first, hf1 = 1 - hf0;
                 __syncwarp();
                 tc_fence_after();
                 if (elect_one()) {
-                    const uint32_t d = tmem + kTmColS + kTmHeads * bi;
 #pragma unroll
-                    for (int kk = 0; kk < ROLAQ_D_C / 16; ++kk)
-                        umma_ts1(d, tmem + kTmColXq + 8 * kk, dq + (uint64_t)((kk * 256) >> 4), kTmIdQk,
-                                 kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < ROLAQ_D_C / 32; ++kk)
+                        umma_ts1(d, tmem + kTmColXq + 8 * (16 * hf0 + kk),
+                                 dq + (uint64_t)(((16 * hf0 + kk) * 256) >> 4), kTmIdQk, kk > 0 ? 1u : 0u);
+                    umma_commit(smem_u32(&sm.xq_free[hf0]));
+                }
+                __syncwarp();
+                mbar_wait(smem_u32(&sm.xq_full[hf1]), (unsigned)(i & 1), &sm.abort);
+                mbar_wait(smem_u32(&sm.full[st]), (unsigned)((i / kTmStages) & 1), &sm.abort);
+                __syncwarp();
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int kk = 0; kk < ROLAQ_D_C / 32; ++kk)
+                        umma_ts1(d, tmem + kTmColXq + 8 * (16 * hf1 + kk),
+                                 dq + (uint64_t)(((16 * hf1 + kk) * 256) >> 4), kTmIdQk, 1u);
                     const uint64_t dk = dkr + (uint64_t)((st * kTmTok * 128) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < ROLAQ_D_R / 16; ++kk)
                         umma_ss1(d, dk + (uint64_t)((kk * 32) >> 4), dqr + (uint64_t)((kk * 256) >> 4), kTmIdRope, 1u);
                     umma_commit(smem_u32(&sm.sfull[bi]));
-                    umma_commit(smem_u32(&sm.xq_free));
+                    umma_commit(smem_u32(&sm.xq_free[hf1]));
                     umma_commit(smem_u32(&sm.pfree[st]));
                 }
                 __syncwarp();
@@ -354,7 +371,7 @@ rolaq_decode_tm(const __grid_constant__ CUtensorMap map_cm, const __grid_constan
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&sm.xp_full[pend_n % kTmXpSlots]));
+                mbar_arrive_lane0(smem_u32(&sm.xp_full[pend_n % kTmXpSlots]));
                 pend_n = -1;
             }
         };
@@ -431,10 +448,8 @@ rolaq_decode_tm(const __grid_constant__ CUtensorMap map_cm, const __grid_constan
                 }
             }
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(smem_u32(&sm.pfree[st]));
-                mbar_arrive(smem_u32(&sm.tbl_free[j % 3]));
-            }
+            mbar_arrive_lane0(smem_u32(&sm.pfree[st]));
+            mbar_arrive_lane0(smem_u32(&sm.tbl_free[j % 3]));
         }
         flush();
     } else if (warp >= kTmTm0) {
@@ -446,10 +461,109 @@ rolaq_decode_tm(const __grid_constant__ CUtensorMap map_cm, const __grid_constan
         const int nslot = args.n_sink + args.n_recent;
         const int recent0 = L - args.n_recent;
         const int t = 32 * q + lane, tp = t >> 6, trow = t & 63;     // token of the tile (S lane)
-        // softmax state (set 0 only): running reference maximum and sum per head
-        float m_ref[kTmHeads], l[kTmHeads];
+        // softmax of this set's eight heads (hb .. hb + 7): running reference maximum and
+        // sum per head; both sets take part, each with its own named barrier
+        constexpr int kH = kTmHeads / 2;
+        const int hb = kH * set;
+        float m_ref[kH], l[kH];
 #pragma unroll
-        for (int h = 0; h < kTmHeads; ++h) { m_ref[h] = -INFINITY; l[h] = 0.f; }
+        for (int h = 0; h < kH; ++h) { m_ref[h] = -INFINITY; l[h] = 0.f; }
+        // softmax of tile i: runs after the token-major x of tile i + 1 is written, so it
+        // overlaps that tile's QK instead of delaying it
+        auto softmax_tile = [&](int i) {
+            const int bi = i & 1;
+            const int pos = (first_page + 2 * i + (t >> 6)) * kPageTok + (t & 63);
+            const bool valid = tm_page_ok(args, b, first_page, T, 2 * i + (t >> 6)) && pos < L;
+            mbar_wait(smem_u32(&sm.sfull[bi]), (unsigned)((i >> 1) & 1), &sm.abort);
+            __syncwarp();
+            tc_fence_after();
+            uint32_t u[kH];
+            tmem_ld8(tmem + lane_base + kTmColS + kTmHeads * bi + hb, u);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            mbar_arrive_lane0(smem_u32(&sm.sfree[bi]));
+            float s[kH];
+            bool up = false;
+#pragma unroll
+            for (int h = 0; h < kH; ++h) {
+                s[h] = valid ? __uint_as_float(u[h]) * args.scale_log2 : -INFINITY;
+                up |= s[h] > m_ref[h] + kRescaleLog2 || (m_ref[h] == -INFINITY && s[h] > -INFINITY);
+            }
+            const bool wup = __any_sync(0xffffffffu, up);
+            if (lane == 0) sm.vote[set][bi][q] = wup ? 1 : 0;
+            named_bar_sync(1 + set, 128);
+            const bool any = (sm.vote[set][bi][0] | sm.vote[set][bi][1] | sm.vote[set][bi][2] | sm.vote[set][bi][3]) != 0;
+            if (any) {
+                // per-head maximum over the tile's 128 tokens
+#pragma unroll
+                for (int h = 0; h < kH; ++h) {
+                    float mx = s[h];
+#pragma unroll
+                    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    if (lane == 0) sm.red[set][q][h] = mx;
+                }
+                named_bar_sync(1 + set, 128);
+                if (q == 0 && lane < kH) {
+                    const int h = hb + lane;
+                    const float tm = fmaxf(fmaxf(sm.red[set][0][lane], sm.red[set][1][lane]),
+                                           fmaxf(sm.red[set][2][lane], sm.red[set][3][lane]));
+                    const float mo = sm.mref[h];
+                    float al = 1.f, mn = mo;
+                    if (tm > mo + kRescaleLog2 || (mo == -INFINITY && tm > -INFINITY)) {
+                        al = (mo == -INFINITY) ? 0.f : ex2(mo - tm);
+                        mn = tm;
+                    }
+                    sm.alpha[h] = al;
+                    sm.mref[h] = mn;
+                }
+                named_bar_sync(1 + set, 128);
+                bool moved = false;
+#pragma unroll
+                for (int h = 0; h < kH; ++h) {
+                    const float al = sm.alpha[hb + h];
+                    m_ref[h] = sm.mref[hb + h];
+                    l[h] *= al;
+                    moved |= al != 1.f;
+                }
+                if (moved && i > 0) {
+                    // O holds PV of tiles 0..i-1: wait for PV(i-1), scale this set's heads in
+                    // this quarter's lanes
+                    mbar_wait(smem_u32(&sm.pvdone[(i - 1) & 1]), (unsigned)(((i - 1) >> 1) & 1), &sm.abort);
+                    __syncwarp();
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int g = 0; g < ROLAQ_GROUPS; ++g) {
+                        uint32_t v[kH];
+                        tmem_ld8(tmem + lane_base + kTmColO + 16 * g + hb, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int h = 0; h < kH; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * sm.alpha[hb + h]);
+                        tmem_st8(tmem + lane_base + kTmColO + 16 * g + hb, v);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                }
+                named_bar_sync(1 + set, 128);  // red / alpha are read by every warp of the set before reuse
+            }
+            // P buffer bi is free once PV(i - 2) has completed
+            if (i >= 2) mbar_wait(smem_u32(&sm.pvdone[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
+            uint32_t pw[kH / 2];
+#pragma unroll
+            for (int h2 = 0; h2 < kH / 2; ++h2) {
+                const float p0 = (m_ref[2 * h2] == -INFINITY) ? 0.f : ex2(s[2 * h2] - m_ref[2 * h2]);
+                const float p1 = (m_ref[2 * h2 + 1] == -INFINITY) ? 0.f : ex2(s[2 * h2 + 1] - m_ref[2 * h2 + 1]);
+                l[2 * h2] += p0;
+                l[2 * h2 + 1] += p1;
+                pw[h2] = pack_f16(p0, p1);
+            }
+            // row t of P: heads 0-7 in 16-byte chunk 0, heads 8-15 in chunk 1 (32-byte swizzle)
+            *reinterpret_cast<uint4*>(sm.P[bi] + t * 32 + ((set ^ ((t >> 2) & 1)) << 4)) =
+                make_uint4(pw[0], pw[1], pw[2], pw[3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            mbar_arrive_lane0(smem_u32(&sm.pready[bi]));
+        };
         for (int i = 0; i < nt; ++i) {
             const int st = i % kTmStages;
             mbar_wait(smem_u32(&sm.full[st]), (unsigned)((i / kTmStages) & 1), &sm.abort);
@@ -462,7 +576,7 @@ rolaq_decode_tm(const __grid_constant__ CUtensorMap map_cm, const __grid_constan
                 const int slot = pos < args.n_sink ? pos : args.n_sink + pos % args.n_recent;
                 prow = args.prot + ((size_t)b * nslot + slot) * ROLAQ_D_C;
             }
-            if (i >= 1) mbar_wait(smem_u32(&sm.xq_free), (unsigned)((i - 1) & 1), &sm.abort);
+            if (i >= 1) mbar_wait(smem_u32(&sm.xq_free[set]), (unsigned)((i - 1) & 1), &sm.abort);
             __syncwarp();
             tc_fence_after();
 #pragma unroll 1
@@ -478,136 +592,38 @@ rolaq_decode_tm(const __grid_constant__ CUtensorMap map_cm, const __grid_constan
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(smem_u32(&sm.xq_full));
-                mbar_arrive(smem_u32(&sm.tbl_full[i % 3]));
-                mbar_arrive(smem_u32(&sm.pfree[st]));
-            }
-            if (set == 0) {
-                // ---- softmax of tile i (the scores need QK(i), which also frees x) ----
-
-            const int bi = i & 1;
-            const int pos = (first_page + 2 * i + (t >> 6)) * kPageTok + (t & 63);
-            const bool valid = tm_page_ok(args, b, first_page, T, 2 * i + (t >> 6)) && pos < L;
-            mbar_wait(smem_u32(&sm.sfull[bi]), (unsigned)((i >> 1) & 1), &sm.abort);
-            __syncwarp();
-            tc_fence_after();
-            uint32_t u[16];
-            tmem_ld16(tmem + lane_base + kTmColS + kTmHeads * bi, u);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.sfree[bi]));
-            float s[kTmHeads];
-            bool up = false;
-#pragma unroll
-            for (int h = 0; h < kTmHeads; ++h) {
-                s[h] = valid ? __uint_as_float(u[h]) * args.scale_log2 : -INFINITY;
-                up |= s[h] > m_ref[h] + kRescaleLog2 || (m_ref[h] == -INFINITY && s[h] > -INFINITY);
-            }
-            const bool wup = __any_sync(0xffffffffu, up);
-            if (lane == 0) sm.vote[bi][q] = wup ? 1 : 0;
-            named_bar_sync(1, 128);
-            const bool any = (sm.vote[bi][0] | sm.vote[bi][1] | sm.vote[bi][2] | sm.vote[bi][3]) != 0;
-            if (any) {
-                // per-head maximum over the tile's 128 tokens
-#pragma unroll
-                for (int h = 0; h < kTmHeads; ++h) {
-                    float mx = s[h];
-#pragma unroll
-                    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                    if (lane == 0) sm.red[q][h] = mx;
-                }
-                named_bar_sync(1, 128);
-                if (q == 0 && lane < kTmHeads) {
-                    const int h = lane;
-                    const float tm = fmaxf(fmaxf(sm.red[0][h], sm.red[1][h]), fmaxf(sm.red[2][h], sm.red[3][h]));
-                    const float mo = sm.mref[h];
-                    float al = 1.f, mn = mo;
-                    if (tm > mo + kRescaleLog2 || (mo == -INFINITY && tm > -INFINITY)) {
-                        al = (mo == -INFINITY) ? 0.f : ex2(mo - tm);
-                        mn = tm;
-                    }
-                    sm.alpha[h] = al;
-                    sm.mref[h] = mn;
-                }
-                named_bar_sync(1, 128);
-                bool moved = false;
-#pragma unroll
-                for (int h = 0; h < kTmHeads; ++h) {
-                    const float al = sm.alpha[h];
-                    m_ref[h] = sm.mref[h];
-                    l[h] *= al;
-                    moved |= al != 1.f;
-                }
-                if (moved && i > 0) {
-                    // O holds PV of tiles 0..i-1: wait for PV(i-1), scale this quarter's lanes
-                    mbar_wait(smem_u32(&sm.pvdone[(i - 1) & 1]), (unsigned)(((i - 1) >> 1) & 1), &sm.abort);
-                    __syncwarp();
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int g = 0; g < ROLAQ_GROUPS; ++g) {
-                        uint32_t v[16];
-                        tmem_ld16(tmem + lane_base + kTmColO + 16 * g, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int h = 0; h < kTmHeads; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * sm.alpha[h]);
-                        tmem_st16(tmem + lane_base + kTmColO + 16 * g, v);
-                    }
-                    tmem_st_wait();
-                    tc_fence_before();
-                }
-                named_bar_sync(1, 128);        // red / alpha are read by every softmax warp before reuse
-            }
-            // P buffer bi is free once PV(i - 2) has completed
-            if (i >= 2) mbar_wait(smem_u32(&sm.pvdone[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
-            uint32_t pw[8];
-#pragma unroll
-            for (int h2 = 0; h2 < kTmHeads / 2; ++h2) {
-                const float p0 = (m_ref[2 * h2] == -INFINITY) ? 0.f : ex2(s[2 * h2] - m_ref[2 * h2]);
-                const float p1 = (m_ref[2 * h2 + 1] == -INFINITY) ? 0.f : ex2(s[2 * h2 + 1] - m_ref[2 * h2 + 1]);
-                l[2 * h2] += p0;
-                l[2 * h2 + 1] += p1;
-                pw[h2] = pack_f16(p0, p1);
-            }
-            uint8_t* prow = sm.P[bi] + t * 32;
-            const int sw = (t >> 2) & 1;
-            *reinterpret_cast<uint4*>(prow + ((0 ^ sw) << 4)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
-            *reinterpret_cast<uint4*>(prow + ((1 ^ sw) << 4)) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.pready[bi]));
-                    }
+            mbar_arrive_lane0(smem_u32(&sm.xq_full[set]));
+            mbar_arrive_lane0(smem_u32(&sm.tbl_full[i % 3]));
+            mbar_arrive_lane0(smem_u32(&sm.pfree[st]));
+            if (i >= 1) softmax_tile(i - 1);
         }
-        if (set == 0) {
-
-        // ---- this item's partial: O (rows = channel lanes), per-head (m, l) ----------
+        if (nt > 0) softmax_tile(nt - 1);
+        // ---- this item's partial: O (rows = channel lanes), per-head (m, l), this set's heads
         if (nt > 0) mbar_wait(smem_u32(&sm.pvdone[(nt - 1) & 1]), (unsigned)(((nt - 1) >> 1) & 1), &sm.abort);
         __syncwarp();
         tc_fence_after();
         const int ch_in_group = 32 * q + 4 * (lane & 7) + (lane >> 3);
 #pragma unroll 1
         for (int g = 0; g < ROLAQ_GROUPS; ++g) {
-            uint32_t v[16];
-            tmem_ld16(tmem + lane_base + kTmColO + 16 * g, v);
+            uint32_t v[kH];
+            tmem_ld8(tmem + lane_base + kTmColO + 16 * g + hb, v);
             tmem_ld_wait();
-            float* dst = args.ws_o + ((size_t)blockIdx.x * args.heads + h0) * ROLAQ_D_C + 128 * g + ch_in_group;
+            float* dst = args.ws_o + ((size_t)blockIdx.x * args.heads + h0 + hb) * ROLAQ_D_C + 128 * g + ch_in_group;
 #pragma unroll
-            for (int h = 0; h < kTmHeads; ++h) dst[(size_t)h * ROLAQ_D_C] = __uint_as_float(v[h]);
+            for (int h = 0; h < kH; ++h) dst[(size_t)h * ROLAQ_D_C] = __uint_as_float(v[h]);
         }
 #pragma unroll
-        for (int h = 0; h < kTmHeads; ++h) {
+        for (int h = 0; h < kH; ++h) {
             float v = l[h];
 #pragma unroll
             for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) sm.red[q][h] = v;
+            if (lane == 0) sm.red[set][q][h] = v;
         }
-        named_bar_sync(1, 128);
-        if (q == 0 && lane < kTmHeads) {
-            const int h = lane;
-            args.ws_ml[(size_t)blockIdx.x * args.heads + h0 + h] =
-                make_float2(sm.mref[h], (sm.red[0][h] + sm.red[1][h]) + (sm.red[2][h] + sm.red[3][h]));
-        }
+        named_bar_sync(1 + set, 128);
+        if (q == 0 && lane < kH) {
+            args.ws_ml[(size_t)blockIdx.x * args.heads + h0 + hb + lane] =
+                make_float2(sm.mref[hb + lane], (sm.red[set][0][lane] + sm.red[set][1][lane]) +
+                                                    (sm.red[set][2][lane] + sm.red[set][3][lane]));
         }
     }
     tc_fence_before();
