@@ -40,7 +40,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # decode kernel sources it was taken on.  The bench reports it only while those sources
 # are unchanged, and null otherwise.
 DECODE_TRAFFIC = {"sources_sha256": None, "bytes_per_launch": None}
-DECODE_SOURCES = ("common.cuh", "decode.cuh", "decode_tm.cuh")
+DECODE_SOURCES = ("common.cuh", "decode.cuh")
 
 
 def decode_sources_sha256():

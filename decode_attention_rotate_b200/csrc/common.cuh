@@ -92,29 +92,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity, volatil
     return false;
 }
 
-// Bounded wait for whichever of two barriers completes its phase first: 0 or 1, or -1
-// when the CTA aborts or the wait gives up.  Called by a whole warp; lane 0 decides.
-__device__ __forceinline__ int mbar_wait_either(uint32_t bar0, uint32_t bar1, unsigned parity,
-                                                volatile int* abort) {
-    int which = -1;
-    if ((threadIdx.x & 31) == 0) {
-        const long long t0 = clock64();
-        for (unsigned it = 0;; ++it) {
-            if (mbar_try_wait(bar0, parity)) { which = 0; break; }
-            if (mbar_try_wait(bar1, parity)) { which = 1; break; }
-            if ((it & 15u) == 15u) {
-                if (*abort) break;
-                if (clock64() - t0 > kWaitCycles) {
-                    *abort = 1;
-                    raise_status(ROLAQ_STATUS_TIMEOUT);
-                    break;
-                }
-            }
-        }
-    }
-    return __shfl_sync(0xffffffffu, which, 0);
-}
-
 // ------------------------------------------------------- bulk tensor copies -----
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
@@ -194,18 +171,6 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 __device__ __forceinline__ void tmem_st_wait() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-// 32 lanes x 8 columns of 32-bit words, one lane per thread.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&u)[8]) {
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
-                 : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&u)[8]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
-                 :: "r"(taddr), "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]),
-                    "r"(u[7])
-                 : "memory");
 }
 // 16 lanes x 16 columns, twice: threads 0-15 write lanes 0-15 of the quarter at `taddr`,
 // threads 16-31 the same lanes 64 columns further.
@@ -295,25 +260,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 }
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(addr), "f"(v) : "memory");
-}
-
-// 16 lanes x 256 bits (8 columns): thread i holds lanes i/4 and i/4 + 8 of the 16-lane
-// block at `taddr`, columns 2(i%4) and 2(i%4) + 1 (registers: (lane i/4, column 2(i%4)),
-// (i/4, 2(i%4)+1), (i/4+8, 2(i%4)), (i/4+8, 2(i%4)+1)).
-__device__ __forceinline__ void tmem_st16x256(uint32_t taddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1,%2,%3,%4};"
-                 :: "r"(taddr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-// Shared-memory matrix descriptor of an MN-major operand with the 32-byte swizzle: rows of
-// 32 bytes (16 two-byte elements along M or N), 8-row groups `sbo` bytes apart along K.
-__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr, uint32_t sbo) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) |
-           (1ull << 46) | (6ull << 61);
 }
 
 // 128-byte swizzle of a (row, byte) position inside a 1024-byte aligned tile:

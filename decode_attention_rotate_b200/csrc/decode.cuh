@@ -426,7 +426,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                 load_page(sm, &map_page, args, page_id(args, b, page_of(k)), k);
             }
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMAs ----
+        // ---------------------------------------------------------------- QK issue ----
         // The whole warp runs this loop (warp-uniform descriptors); each MMA and commit is
         // issued by one elected lane.
         {
@@ -435,40 +435,15 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             const uint64_t dqc = smem_desc(smem_u32(sm.qc), 128, 64 * 128, 0);
             const uint64_t dqr = smem_desc(smem_u32(sm.qr), 128, 8 * 128, 0);
             // (buffers of one kind are contiguous: buffer n starts n * size bytes later)
-            const uint64_t dxk = smem_desc(smem_u32(sm.x[0]), 16, 1024, 2);          // K-major view (QK)
-            const uint64_t dxm = smem_desc(smem_u32(sm.x[0]), kXAtom, 1024, 2);      // MN-major view (PV)
-            const uint64_t dp = smem_desc(smem_u32(sm.P[0]), 128, 1024, 0);
             const uint64_t dkr = smem_desc(smem_u32(sm.stage[0]) + kKrRow * 128, 16, 1024, 2);
-            auto pv = [&](int j) {
-                const int bj = j & 1;
-                mbar_wait(smem_u32(&sm.pready[bj]), (unsigned)((j >> 1) & 1), &sm.abort);
-                __syncwarp();
-                tc_fence_after();
-                const uint64_t da = dxm + (uint64_t)(bj * (kXTile >> 4)), db = dp + (uint64_t)(bj * (sizeof(sm.P[0]) >> 4));
-                const uint32_t first = j > 0 ? 1u : 0u;
-                if (elect_one()) {
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-#pragma unroll
-                        for (int ks = 0; ks < kPageTok / 16; ++ks)
-                            umma_ss1(tmem + kOCol + HC * g, da + (uint64_t)((2 * g * kXAtom + ks * 2048) >> 4),
-                                     db + (uint64_t)((ks * 256) >> 4), kIdPv, ks > 0 ? 1u : first);
-                        if (g == 1) umma_commit(smem_u32(&sm.xfree[bj][0]));   // groups 0-1 read
-                    }
-                    umma_commit(smem_u32(&sm.xfree[bj][1]));
-                }
-                __syncwarp();
-            };
             for (int i = 0; i < T; ++i) {
                 const int bi = i & 1, st = i % kStages;
                 if (i >= 2) mbar_wait(smem_u32(&sm.sfree[bi]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
-                const uint64_t da = dxk + (uint64_t)(bi * (kXTile >> 4));
                 const uint64_t dk = dkr + (uint64_t)(st * (ROLAQ_PAGE_BYTES >> 4));
                 const uint32_t d = tmem + kSCol + HC * bi;
                 // QK from the token-major x in tensor memory (M = 64: token r in lane
                 // 32 (r / 16) + r % 16), channel groups 0-1 (K steps 0..15) as soon as that
                 // half is written, then groups 2-3 and the RoPE keys
-                (void)da;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     mbar_wait(smem_u32(&sm.xq_full[hf]), (unsigned)(i & 1), &sm.abort);
@@ -493,9 +468,40 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                     }
                     __syncwarp();
                 }
-                if (i >= 1) pv(i - 1);
             }
-            if (T > 0) pv(T - 1);
+        }
+    } else if (warp == 2) {
+        // ---------------------------------------------------------------- PV issue ----
+        // PV has its own warp, so the PV of page i - 1 never waits behind the QK of page i
+        // (different accumulators and operands; each issuing thread's commits track only its
+        // own products).
+        {
+            // x tiles read MN-major (buffers of one kind are contiguous)
+            const uint64_t dxm = smem_desc(smem_u32(sm.x[0]), kXAtom, 1024, 2);
+            const uint64_t dp = smem_desc(smem_u32(sm.P[0]), 128, 1024, 0);
+            auto pv = [&](int j) {
+                const int bj = j & 1;
+                mbar_wait(smem_u32(&sm.pready[bj]), (unsigned)((j >> 1) & 1), &sm.abort);
+                mbar_wait(smem_u32(&sm.xready[bj][0]), (unsigned)((j >> 1) & 1), &sm.abort);
+                mbar_wait(smem_u32(&sm.xready[bj][1]), (unsigned)((j >> 1) & 1), &sm.abort);
+                __syncwarp();
+                tc_fence_after();
+                const uint64_t da = dxm + (uint64_t)(bj * (kXTile >> 4)), db = dp + (uint64_t)(bj * (sizeof(sm.P[0]) >> 4));
+                const uint32_t first = j > 0 ? 1u : 0u;
+                if (elect_one()) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+#pragma unroll
+                        for (int ks = 0; ks < kPageTok / 16; ++ks)
+                            umma_ss1(tmem + kOCol + HC * g, da + (uint64_t)((2 * g * kXAtom + ks * 2048) >> 4),
+                                     db + (uint64_t)((ks * 256) >> 4), kIdPv, ks > 0 ? 1u : first);
+                        if (g == 1) umma_commit(smem_u32(&sm.xfree[bj][0]));   // groups 0-1 read
+                    }
+                    umma_commit(smem_u32(&sm.xfree[bj][1]));
+                }
+                __syncwarp();
+            };
+            for (int j = 0; j < T; ++j) pv(j);
         }
     } else if (warp >= kDqWarp0) {
         // ------------------------------------------------------------- dequant ----

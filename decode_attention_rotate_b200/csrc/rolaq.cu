@@ -7,7 +7,6 @@
 
 #include "common.cuh"
 #include "decode.cuh"
-#include "decode_tm.cuh"
 #include "project.cuh"
 #include "quantize.cuh"
 
@@ -16,9 +15,6 @@ using namespace rolaq;
 namespace {
 
 constexpr int kVersion = 100;   // 0.1.0
-// The tensor-memory-operand decode (decode_tm.cuh) takes 16-head chunks once it beats the
-// shared-memory decode on the long-context workload; until then both are built.
-constexpr bool kDecodeTm = false;
 constexpr int kMaxDevices = 64;
 
 int device_sms(int dev) {
@@ -307,19 +303,7 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
                                         (size_t)items_cap * heads * ROLAQ_D_C * sizeof(float));
 
     cudaStream_t s = (cudaStream_t)stream;
-    if (heads % 32 != 0 && kDecodeTm) {
-        // 16 heads per CTA, both tensor-core A operands in tensor memory
-        CUtensorMap map_cm, map_kr;
-        if (!encode_2d(&map_cm, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache->pages_dev, 128, rows, 128, 128, kTmCmRows,
-                       CU_TENSOR_MAP_SWIZZLE_128B) ||
-            !encode_2d(&map_kr, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache->pages_dev, 128, rows, 128, 128, kTmKrRows,
-                       CU_TENSOR_MAP_SWIZZLE_128B))
-            return ROLAQ_ECUDA;
-        const size_t smem = sizeof(TmSmem) + 1024;
-        static bool attr_done[kMaxDevices] = {false};
-        set_smem_limit_once(rolaq_decode_tm, smem, attr_done);
-        rolaq_decode_tm<<<dim3(items_cap, heads / kTmHeads), kTmThreads, smem, s>>>(map_cm, map_kr, a);
-    } else if (heads % 32 == 0) {
+    if (heads % 32 == 0) {
         // 32 heads per CTA (twice the work per tensor-core instruction and per
         // dequantised tile)
         const size_t smem = sizeof(DecodeSmem<32>) + 1024;
