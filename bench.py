@@ -1,9 +1,9 @@
 #!/usr/bin/env python
 """Benchmark of the 2-bit rotated MLA cache hot path on B200.
 
-Step = one decode step of the long-context serving shape: for each of 27 layers, append
-one new token per request (write path: rotate, quantize, pack) and run the absorbed-MLA
-decode over 4 requests x 262,144 cached tokens at 16 heads (read path).  The cache of a
+Step = one decode step of the long-context serving shape: for each of 27 layers, one call
+that appends one new token per request (write path: rotate, quantize, pack) and runs the
+absorbed-MLA decode over 4 requests x 262,144 cached tokens at 16 heads (read path).  The cache of a
 step is 8.15 GB, far larger than L2, so no flush is needed between steps.  value = cache
 GB/s over the whole step (all ranks; replicas are independent, weak scaling).
 Also measured: the prefill write path on 65,536 tokens x 27 layers (tokens/s), and the
@@ -212,12 +212,11 @@ def cpu_oracle_decode_rate(w, layers, budget_s=12.0):
 def run_ours(args, rank, world, dev):
     w = W.DECODE_4x256K_27L
     layers = build_decode_workload(w, dev)
-    ws = torch.empty(R.decode_workspace_bytes(w.batch, w.heads), dtype=torch.uint8, device=dev)
+    ws = torch.empty(R.decode_append_workspace_bytes(w.batch, w.heads), dtype=torch.uint8, device=dev)
     lens = torch.as_tensor(w.seq_lens, dtype=torch.int32, device=dev)
     # the token appended each step overwrites the last position, so every step decodes
-    # the same 262,144 tokens per request
-    new_req = torch.arange(w.batch, dtype=torch.int32, device=dev)
-    new_pos = (lens - 1).clone()
+    # the same 262,144 tokens per request; the append runs inside the decode call (the
+    # split kernel rotates the new tokens, the merge kernel stores them and adds their term)
     new_c = [W.latent_device(w, l, w.batch, dev, stream=9000) for l in range(w.layers)]
     new_kr = [W.rope_key_device(w, l, w.batch, dev, stream=9001) for l in range(w.layers)]
     stream = torch.cuda.current_stream()
@@ -225,10 +224,10 @@ def run_ours(args, rank, world, dev):
 
     def step(record):
         for l, lay in enumerate(layers):
-            R.quantize_append(lay.cache, lay.params, lay.R_split, new_c[l], new_kr[l], new_req, new_pos)
             if record:
                 ev[l][0].record(stream)
-            R.decode_attn(lay.cache, lay.params, lay.q_c, lay.q_r, lens, SM_SCALE, lay.out, lay.lse, ws)
+            R.decode_attn_append(lay.cache, lay.params, lay.R_split, new_c[l], new_kr[l], lay.q_c, lay.q_r, lens,
+                                 SM_SCALE, lay.out, lay.lse, ws)
             if record:
                 ev[l][1].record(stream)
 
@@ -274,8 +273,8 @@ def run_ours(args, rank, world, dev):
             hc, hkr, hqc, hqr = host_in[l]
             c.copy_(hc, non_blocking=True); kr.copy_(hkr, non_blocking=True)
             qc.copy_(hqc, non_blocking=True); qr.copy_(hqr, non_blocking=True)
-            R.quantize_append(lay.cache, lay.params, lay.R_split, c, kr, new_req, new_pos)
-            R.decode_attn(lay.cache, lay.params, qc, qr, lens, SM_SCALE, lay.out, lay.lse, ws)
+            R.decode_attn_append(lay.cache, lay.params, lay.R_split, c, kr, qc, qr, lens, SM_SCALE, lay.out,
+                                 lay.lse, ws)
             host_out[l][0].copy_(lay.out, non_blocking=True)
             host_out[l][1].copy_(lay.lse, non_blocking=True)
 
@@ -301,12 +300,15 @@ def run_ours(args, rank, world, dev):
     bf16_stats = _guarded(bench_bf16_baseline, args, dev, world, w, dec_ms)
     bf16_stats["ours_all_protected"] = bench_all_protected(args, dev, dec_ms)
     cfg_stats = _guarded(bench_configs, args, dev)
+    sweep_stats = _guarded(bench_tau_sweep, dev)
     proj_stats = [_guarded(bench_projections, args, dev, world, w.batch, w.heads),
                   _guarded(bench_projections, args, dev, world, W.PAGED_H128.batch, W.PAGED_H128.heads)]
     clocks = sampler.stop()     # sampled across the timed regions
 
     hbm, bf16, src = peaks()
-    dec_bytes = w.total_tokens * R.TOKEN_BYTES
+    # the cache, plus what the fused append must read and write once per call: the rotation
+    # planes, the new tokens' latents and RoPE keys, and their records
+    dec_bytes = w.total_tokens * R.TOKEN_BYTES + R.RSPLIT_BYTES + w.batch * (1024 + 128 + R.TOKEN_BYTES)
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -319,16 +321,17 @@ def run_ours(args, rank, world, dev):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "traffic": decode_traffic(),
-                     "kernel": "decode call (split + merge launches); traffic: split kernel",
+                     "kernel": "fused append + decode call (split + merge launches); traffic: split kernel",
                      "peak_source": src,
                      "bytes_per_launch": dec_bytes, "ms_per_launch": round(dec_ms, 4),
                      "frac_of_8tbs": round(achieved / 8000.0, 4)},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
-        "gpu_launches": args.steps * w.layers * 3,
+        "gpu_launches": args.steps * w.layers * 2,
         "quantize": q_stats,
         "bf16_baseline": bf16_stats,
         "projections": proj_stats,
+        "tau_sweep": sweep_stats,
         "other_workloads": cfg_stats,
         "clocks": clocks,
     }
@@ -382,6 +385,71 @@ def bench_quantize(args, dev, world):
                          "executed_flops_factor": 3, "peak_source": src},
             "hbm": {"achieved": round(bytes_ / (per_launch_ms * 1e-3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
                     "frac": round(bytes_ / (per_launch_ms * 1e-3) / 1e9 / hbm, 4)}}
+
+
+# ------------------------------------------------------------ threshold sweep ----
+# The write path at several thresholds tau, each with its coupled gain g(tau) from the
+# library: every token of one 8,192-token request is also kept as a protected bf16 copy,
+# so the stored codes, the stored statistics and bf16(y) all come from the same call.
+# Reported per tau: the outer-code fraction (and 2(1 - Phi(tau)) for a normal
+# coordinate), the fraction of codes that differ from those at the Lloyd-Max threshold,
+# and the reconstruction response sum((x - mean)(y - mean)) / sum((y - mean)^2) with the
+# coupled gain (unit response is the aim) and at gain 1, plus the normalised error.
+SWEEP_TAUS = (0.85, 0.88, 0.91, 0.94, 0.9816, 1.02, 1.06, 1.10)
+LLOYD_MAX_TAU = 0.9816
+
+
+def unpack_codes(pages, n):
+    """Codes [n, 512] of a request laid out on consecutive pages (byte b of a token holds
+    coordinates 4b..4b+3, coordinate j at bits 2(j % 4))."""
+    pg = pages.reshape(-1, R.PAGE_BYTES)[:, :R.PAGE_TOKENS * R.CODE_BYTES]
+    b = pg.reshape(-1, R.CODE_BYTES)[:n].astype(np.uint8)
+    return np.stack([(b >> (2 * j)) & 3 for j in range(4)], axis=2).reshape(n, R.D_C)
+
+
+def unpack_meta(pages, n):
+    off = R.PAGE_TOKENS * R.CODE_BYTES
+    pg = pages.reshape(-1, R.PAGE_BYTES)[:, off:off + R.PAGE_TOKENS * R.META_BYTES]
+    return np.ascontiguousarray(pg).view(np.float32).reshape(-1, R.GROUPS, 2)[:n].astype(np.float64)
+
+
+def bench_tau_sweep(dev, n=8192):
+    w = W.Workload("tau_sweep_8k", 1, (n,), 16, n_sink=n, seed=4250)
+    pt = torch.as_tensor(W.page_table(w))
+    Rs = R.prepare_rotation(torch.as_tensor(W.rotation(w.seed)).to(dev))
+    c = W.latent_device(w, 0, n, dev)
+    kr = W.rope_key_device(w, 0, n, dev)
+    req = torch.zeros(n, dtype=torch.int32, device=dev)
+    pos = torch.arange(n, dtype=torch.int32, device=dev)
+    rows, ref = [], None
+    runs = {}
+    for tau in SWEEP_TAUS:
+        gain, kappa1 = R.coupled_gain(tau)
+        p = R.layer_params_init(tau, gain)
+        cache = R.PagedCache(int(pt.max()) + 1, pt, n_sink=n, device=dev)
+        R.quantize_append(cache, p, Rs, c, kr, req, pos)
+        torch.cuda.synchronize()
+        pages = cache.pages.cpu().numpy()
+        y = cache.prot[0].float().cpu().numpy().astype(np.float64).reshape(n, R.GROUPS, R.GROUP)
+        runs[tau] = (unpack_codes(pages, n), unpack_meta(pages, n), y, p, gain, kappa1)
+    ref = runs[LLOYD_MAX_TAU][0]
+    for tau in SWEEP_TAUS:
+        codes, meta, y, p, gain, kappa1 = runs[tau]
+        lev = np.array([-p.level_b, -p.level_a, p.level_a, p.level_b], dtype=np.float64)
+        mu, scale = meta[:, :, 0:1], meta[:, :, 1:2]
+        xc = scale * lev[codes.reshape(n, R.GROUPS, R.GROUP)]        # x - mean, coupled gain
+        yc = y - mu
+        den = float((yc * yc).sum())
+        resp = float((xc * yc).sum()) / den
+        rows.append({"tau": tau, "gain": round(gain, 6), "kappa_gain1": round(kappa1, 6),
+                     "outer_code_frac": round(float(np.isin(codes, (0, 3)).mean()), 5),
+                     "outer_frac_normal": round(1.0 - math.erf(tau / math.sqrt(2.0)), 5),
+                     "code_flip_frac_vs_lloyd_max": round(float((codes != ref).mean()), 5),
+                     "response": round(resp, 5), "response_gain1": round(resp / gain, 5),
+                     "nmse": round(float(((xc - yc) ** 2).sum()) / den, 5),
+                     "nmse_gain1": round(float(((xc / gain - yc) ** 2).sum()) / den, 5)})
+    return {"workload": w.name, "tokens": n, "lloyd_max_tau": LLOYD_MAX_TAU,
+            "y_source": "bf16 side-store copy written by the same call", "rows": rows}
 
 
 def capture_graph(fn):
@@ -597,6 +665,9 @@ def run_case(args, dev):
     if args.case == "protected":
         print(json.dumps({"case": "protected", "result": bench_all_protected(args, dev, float("nan"))}), flush=True)
         return
+    if args.case == "sweep":
+        print(json.dumps({"case": "sweep", "result": bench_tau_sweep(dev)}), flush=True)
+        return
     if args.case == "configs":
         print(json.dumps({"case": "configs", "results": bench_configs(args, dev)}), flush=True)
         return
@@ -731,7 +802,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["decode", "quantize", "project", "configs", "protected"], default=None,
+    ap.add_argument("--case", choices=["decode", "quantize", "project", "configs", "protected", "sweep"], default=None,
                     help="run one small single-kernel case (for ncu captures) instead of the bench")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 1)

@@ -27,6 +27,14 @@
 //                     (a vote in the common case), in which case O is rescaled before
 //                     the next PV; P goes to shared memory as the fp16 B operand.
 // Kernel B (rolaq_decode_merge): log-sum-exp merge of the per-item partials.
+//
+// Fused append (one new token per request at position L - 1, the per-step write of a
+// serving decode): in kernel A the otherwise idle warp 3 of every CTA of head chunk 0
+// computes a slice of the new tokens' rotated coordinates y = c . R into the workspace,
+// while the item pages exclude position L - 1 (the plan covers L - 1 tokens; the
+// protected window still counts L).  Kernel B, which runs after A, completes the append
+// for its request (group statistics, codes, the page record and side-store row, written
+// by the head-0 CTA) and adds the new token's term to the merge.
 #pragma once
 #include "common.cuh"
 
@@ -65,6 +73,26 @@ struct DecodeArgs {
     int target_items;
     float* ws_o;                 // [items][heads][512]  sum_t 2^(s_t - m) x_t
     float2* ws_ml;               // [items][heads]       (m (log2 units), sum_t 2^(s_t - m))
+    // fused append (append = 1): new token of request b at position seq_lens[b] - 1
+    int append;
+    const __nv_bfloat16* app_R;  // rotation planes [3][512][512] (row = output coordinate)
+    const __nv_bfloat16* app_c;  // new content latents [batch][512]
+    float* ws_y;                 // [batch][512] their rotated coordinates
+};
+
+// What the merge needs to complete a fused append.  y == nullptr: no append.
+struct AppendArgs {
+    const float* y;              // [batch][512] rotated coordinates of the new tokens
+    const __nv_bfloat16* k_r;    // [batch][64] their RoPE keys
+    const __nv_bfloat16* q;      // [batch][heads][512] rotated content queries
+    const __nv_bfloat16* qr;     // [batch][heads][64]
+    float scale_log2, tau, gain, level_a, level_b;
+    uint8_t* pages;
+    const int32_t* page_table;
+    int64_t num_pages;
+    int max_pages;
+    __nv_bfloat16* prot;         // [batch][n_sink + n_recent][512] or null
+    int n_sink, n_recent;
 };
 
 template <int HC>
@@ -105,23 +133,28 @@ static_assert(sizeof(DecodeSmem<32>) + 1024 <= 227 * 1024, "decode shared memory
 // values.
 struct PlanInfo { int b, first_page, n_pages, n_items, item_offset, chunk; };
 
-__device__ __forceinline__ int plan_items(const int32_t* seq_lens, int batch, int chunk) {
+// app = 1 (fused append): the items cover L - 1 tokens of a request of length L.
+__device__ __forceinline__ int plan_pages(const int32_t* seq_lens, int b, int app) {
+    return (max(seq_lens[b] - app, 0) + kPageTok - 1) / kPageTok;
+}
+
+__device__ __forceinline__ int plan_items(const int32_t* seq_lens, int batch, int chunk, int app) {
     const int lane = threadIdx.x & 31;
     int items = 0;
     for (int b = lane; b < batch; b += 32) {
-        const int pages = (max(seq_lens[b], 0) + kPageTok - 1) / kPageTok;
+        const int pages = plan_pages(seq_lens, b, app);
         items += (pages + chunk - 1) / chunk;
     }
     for (int o = 16; o; o >>= 1) items += __shfl_xor_sync(0xffffffffu, items, o);
     return items;
 }
 
-__device__ __forceinline__ int plan_chunk(const int32_t* seq_lens, int batch, int target) {
+__device__ __forceinline__ int plan_chunk(const int32_t* seq_lens, int batch, int target, int app) {
     const int lane = threadIdx.x & 31;
     long long total = 0;
     int max_pages = 0;
     for (int b = lane; b < batch; b += 32) {
-        const int pages = (max(seq_lens[b], 0) + kPageTok - 1) / kPageTok;
+        const int pages = plan_pages(seq_lens, b, app);
         total += pages;
         max_pages = max(max_pages, pages);
     }
@@ -133,11 +166,11 @@ __device__ __forceinline__ int plan_chunk(const int32_t* seq_lens, int batch, in
     // ragged lengths can leave more items than `target` (a second, mostly idle wave);
     // with chunk = max_pages every non-empty request is one item, so when batch <=
     // target a fitting chunk exists: binary search for the smallest
-    if (batch <= target && max_pages > c && plan_items(seq_lens, batch, c) > target) {
+    if (batch <= target && max_pages > c && plan_items(seq_lens, batch, c, app) > target) {
         int lo = c + 1, hi = max_pages;
         while (lo < hi) {
             const int mid = lo + (hi - lo) / 2;
-            if (plan_items(seq_lens, batch, mid) <= target) hi = mid;
+            if (plan_items(seq_lens, batch, mid, app) <= target) hi = mid;
             else lo = mid + 1;
         }
         c = lo;
@@ -147,17 +180,17 @@ __device__ __forceinline__ int plan_chunk(const int32_t* seq_lens, int batch, in
 
 // Locate work item `item` (or request `req` when item < 0).  n_items = total item count.
 __device__ PlanInfo plan_lookup(const int32_t* seq_lens, int batch, int target, int item,
-                                int req) {
+                                int req, int app) {
     const int lane = threadIdx.x & 31;
     PlanInfo pi{-1, 0, 0, 0, 0, 0};
-    const int chunk = plan_chunk(seq_lens, batch, target);
+    const int chunk = plan_chunk(seq_lens, batch, target, app);
     pi.chunk = chunk;
     int base = 0;
     for (int b0 = 0; b0 < batch; b0 += 32) {
         int b = b0 + lane;
         int items = 0, pages = 0;
         if (b < batch) {
-            pages = (max(seq_lens[b], 0) + kPageTok - 1) / kPageTok;
+            pages = plan_pages(seq_lens, b, app);
             items = (pages + chunk - 1) / chunk;
         }
         int incl = items;
@@ -191,26 +224,19 @@ __device__ PlanInfo plan_lookup(const int32_t* seq_lens, int batch, int target, 
     return pi;
 }
 
-// Eight fp16 pairs from one 32-bit word of codes: bytes 0-1 hold 8 codes of token A,
-// bytes 2-3 8 codes of token B (code j of a byte at bits 2j).  r[k][0] = (x_A of code k
-// of byte 0, x_A of code k of byte 1); r[k][1] the same for token B.  A token's lookup
-// pair (lo, hi) holds the low and high bytes of its four fp16 x values, so PRMT nibbles
-// c and c + 4 pick value c: the selector of a byte pair is byte * 0x11 + 0x4040 with the
-// code moved to bits 0-1; __umulhi(m, 0x11 << (16 - s)) does the same for bytes 2-3
-// (every multiplier fits in 32 bits).
-__device__ __forceinline__ void dequant_word2(uint32_t w, uint2 la, uint2 lb, uint32_t (&r)[4][2]) {
-    const uint32_t m0 = w & 0x03030303u;
-    r[0][0] = prmt(la.x, la.y, m0 * 0x11u + 0x4040u);
-    r[0][1] = prmt(lb.x, lb.y, __umulhi(m0, 0x11u << 16) + 0x4040u);
-    const uint32_t m1 = w & 0x0C0C0C0Cu;
-    r[1][0] = prmt(la.x, la.y, (m1 >> 2) * 0x11u + 0x4040u);
-    r[1][1] = prmt(lb.x, lb.y, __umulhi(m1, 0x11u << 14) + 0x4040u);
-    const uint32_t m2 = w & 0x30303030u;
-    r[2][0] = prmt(la.x, la.y, (m2 >> 4) * 0x11u + 0x4040u);
-    r[2][1] = prmt(lb.x, lb.y, __umulhi(m2, 0x11u << 12) + 0x4040u);
-    const uint32_t m3 = w & 0xC0C0C0C0u;
-    r[3][0] = prmt(la.x, la.y, __umulhi(m3, 0x11u << 26) + 0x4040u);
-    r[3][1] = prmt(lb.x, lb.y, __umulhi(m3, 0x11u << 10) + 0x4040u);
+// Sixteen codes of one token (one 32-bit word) into fp16 pairs, one selector per four
+// codes: r[k][0] = (x of byte 0's code k, x of byte 1's code k), r[k][1] the same for
+// bytes 2 and 3.  The lookup pair (lo, hi) holds the low and high bytes of the token's
+// four fp16 values, so selector nibbles (c, c + 4) pick value c; the second pair uses the
+// selector's upper half.
+__device__ __forceinline__ void codes_to_x(uint32_t w, uint2 lut, uint32_t (&r)[4][2]) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t m = (w >> (2 * k)) & 0x03030303u;
+        const uint32_t sel = m * 0x11u + 0x40404040u;
+        r[k][0] = prmt(lut.x, lut.y, sel);
+        r[k][1] = prmt(lut.x, lut.y, sel >> 16);
+    }
 }
 
 // ---- tensor-core operands -----------------------------------------------------
@@ -289,7 +315,7 @@ __device__ __forceinline__ void dequant_tile_part(const uint8_t* pg, int t, int 
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
         uint32_t r[4][2];
-        dequant_word2(cw[w], lut, lut, r);
+        codes_to_x(cw[w], lut, r);
 #pragma unroll
         for (int k = 0; k < 4; ++k) { o[w][k] = r[k][0]; o[w][4 + k] = r[k][1]; }
     }
@@ -337,6 +363,51 @@ __device__ __forceinline__ void tmem_ld_scores(uint32_t taddr, uint32_t (&u)[16]
                  : "r"(taddr));
 }
 
+// Fused append, kernel A part (one warp): output coordinates o = cta, cta + ncta, ... of
+// every new token, y[b][o] = sum_k c[b][k] R[k][o].  Lane l takes inputs 16l .. 16l + 15:
+// the three rotation planes summed in fp32 (smallest first), fma with the latents, then a
+// butterfly over the warp.
+__device__ __forceinline__ void append_rotate(const DecodeArgs& args, int cta, int ncta) {
+    const int lane = threadIdx.x & 31;
+    const size_t plane = (size_t)ROLAQ_D_C * ROLAQ_D_C;
+    for (int o = cta; o < ROLAQ_D_C; o += ncta) {
+        float rk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) rk[i] = 0.f;
+#pragma unroll
+        for (int pl = 2; pl >= 0; --pl) {
+            const uint4* row = reinterpret_cast<const uint4*>(args.app_R + pl * plane + (size_t)o * ROLAQ_D_C);
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {
+                const uint4 u = row[2 * lane + hv];
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    rk[8 * hv + 2 * q] += __uint_as_float(w[q] << 16);
+                    rk[8 * hv + 2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+                }
+            }
+        }
+        for (int b = 0; b < args.batch; ++b) {
+            if (args.seq_lens[b] < 1) continue;
+            const uint4* crow = reinterpret_cast<const uint4*>(args.app_c + (size_t)b * ROLAQ_D_C);
+            float acc = 0.f;
+#pragma unroll
+            for (int hv = 0; hv < 2; ++hv) {
+                const uint4 cu = crow[2 * lane + hv];
+                const uint32_t cw[4] = {cu.x, cu.y, cu.z, cu.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc = fmaf(__uint_as_float(cw[q] << 16), rk[8 * hv + 2 * q], acc);
+                    acc = fmaf(__uint_as_float(cw[q] & 0xFFFF0000u), rk[8 * hv + 2 * q + 1], acc);
+                }
+            }
+            for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (lane == 0) args.ws_y[(size_t)b * ROLAQ_D_C + o] = acc;
+        }
+    }
+}
+
 template <int HC>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
 rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArgs args) {
@@ -352,7 +423,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
     const int hc = blockIdx.y;                 // HC-head chunk
 
     if (warp == 0) {
-        PlanInfo pi = plan_lookup(args.seq_lens, args.batch, args.target_items, (int)blockIdx.x, -1);
+        PlanInfo pi = plan_lookup(args.seq_lens, args.batch, args.target_items, (int)blockIdx.x, -1, args.append);
         if (lane == 0) {
             sm.plan[0] = pi.b;
             sm.plan[1] = pi.first_page;
@@ -382,9 +453,14 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
     }
     __syncthreads();
     const int b = sm.plan[0];
-    if (b < 0) return;                         // item past the end of the plan
+    const bool appender = args.append && blockIdx.y == 0 && warp == 3;
+    if (b < 0) {                               // item past the end of the plan
+        if (appender) append_rotate(args, (int)blockIdx.x, (int)gridDim.x);
+        return;
+    }
     const int first_page = sm.plan[1], T = sm.plan[2];
-    const int L = args.seq_lens[b];
+    const int L = args.seq_lens[b];            // protected window: the last n_recent of L
+    const int Lkv = L - args.append;           // tokens read from the pages
     const int h0 = hc * HC;
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -516,7 +592,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             const int bi = i & 1, st = i % kStages;
             mbar_wait(smem_u32(&sm.full[st]), (unsigned)((i / kStages) & 1), &sm.abort);
             const int pos = page_of(i) * kPageTok + t;
-            const bool valid = sm.valid[st] && pos < L;
+            const bool valid = sm.valid[st] && pos < Lkv;
             const bool prot = valid && protect && (pos < args.n_sink || pos >= L - args.n_recent);
             const __nv_bfloat16* prow = nullptr;
             if (prot) {
@@ -550,6 +626,9 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&sm.xready[bi][hf]));
         }
+    } else if (warp == 3) {
+        // --------------------------------------------------------- fused append ----
+        if (appender) append_rotate(args, (int)blockIdx.x, (int)gridDim.x);
     } else if (warp >= kSoftWarp0) {
         // ------------------------------------------------------------- softmax ----
         // Warp q reads TMEM lane quarter q: S rows 16q..16q+15 (M = 64) in lanes 0..15 with
@@ -585,7 +664,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             bool up = false;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
-                const bool valid = vpage && page_of(i) * kPageTok + rows[j] < L;
+                const bool valid = vpage && page_of(i) * kPageTok + rows[j] < Lkv;
 #pragma unroll
                 for (int e = 0; e < kE; ++e) {
                     const uint32_t raw = u[(e >> 1) * 4 + 2 * j + (e & 1)];
@@ -711,22 +790,113 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
 // w_i = 2^(m_i - max m); lse = (max m + log2(sum w l)) * ln 2.  Warp w takes partials
 // w, w + 16, ...; lane l owns channels 4l + 128j (j = 0..3), so every thread keeps many
 // independent loads in flight; the 16 warp sums are added through shared memory.
+// With a fused append, thread c first finishes channel c of request b's new token:
+// group statistics over the 128 threads of its group (two-pass mean and population std,
+// each a butterfly then the sum of the four warp values), its code, its value x (the
+// bf16 y when the new token is protected, else the fp16 mean + scale * level the decode
+// reads), and the token's score; the head-0 CTA also stores the token's record.  The new
+// token enters the merge as one more partial with m = its score, l = 1, o = x.
 constexpr int kMergeThreads = 512;
+static_assert(kMergeThreads == ROLAQ_D_C, "merge: one thread per latent channel");
+
+__device__ __forceinline__ float merge_group_sum(float v, float (*red)[4], int g, int gw) {
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) red[g][gw] = v;
+    __syncthreads();
+    const float r = (red[g][0] + red[g][1]) + (red[g][2] + red[g][3]);
+    __syncthreads();
+    return r;
+}
+
+__device__ __forceinline__ float merge_block_sum(float v, float* red) {
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    float r = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeThreads / 32; ++w) r += red[w];
+    __syncthreads();
+    return r;
+}
 
 __global__ void __launch_bounds__(kMergeThreads)
 rolaq_decode_merge(const float* __restrict__ ws_o, const float2* __restrict__ ws_ml,
                    const int32_t* seq_lens, int batch, int heads, int target,
-                   float* __restrict__ out, float* __restrict__ lse) {
+                   float* __restrict__ out, float* __restrict__ lse, const AppendArgs app) {
     __shared__ int s_plan[2];
     __shared__ float s_red[kMergeThreads / 32];
+    __shared__ float s_gred[ROLAQ_GROUPS][4];
+    __shared__ uint32_t s_codes[ROLAQ_CODE_BYTES / 4];
     __shared__ float s_M, s_den;
     __shared__ __align__(16) float s_acc[kMergeThreads / 32][ROLAQ_D_C];
     const int b = blockIdx.x, h = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kWarps = kMergeThreads / 32;
+    const int c = threadIdx.x;               // one channel per thread
     if (warp == 0) {
-        PlanInfo pi = plan_lookup(seq_lens, batch, target, -1, b);
+        PlanInfo pi = plan_lookup(seq_lens, batch, target, -1, b, app.y != nullptr ? 1 : 0);
         if (lane == 0) { s_plan[0] = pi.item_offset; s_plan[1] = pi.n_items; }
+    }
+    // ---- the new token (fused append) ----
+    float s_new = -INFINITY, x_new = 0.f;
+    const int L = seq_lens[b];
+    if (app.y != nullptr && L >= 1) {
+        const int g = c >> 7, gw = warp & 3;
+        const float y = app.y[(size_t)b * ROLAQ_D_C + c];
+        const float mean = merge_group_sum(y, s_gred, g, gw) * (1.f / 128.f);
+        const float d = y - mean;
+        const float sd = sqrtf(merge_group_sum(d * d, s_gred, g, gw) * (1.f / 128.f));
+        const float inv = sd > 0.f ? 1.f / sd : 0.f;
+        const float z = d * inv;
+        const uint32_t code = (uint32_t)(z >= -app.tau) + (uint32_t)(z >= 0.f) + (uint32_t)(z >= app.tau);
+        const float scale = app.gain * sd;
+        const int pos = L - 1;
+        const bool prot = app.prot != nullptr && (pos < app.n_sink || app.n_recent > 0);
+        const float yb = __bfloat162float(__float2bfloat16_rn(y));
+        if (prot) {
+            x_new = __half2float(__float2half_rn(yb));
+        } else {
+            const float lev = code == 0 ? -app.level_b : code == 1 ? -app.level_a : code == 2 ? app.level_a : app.level_b;
+            x_new = __half2float(__float2half_rn(fmaf(scale, lev, mean)));
+            if ((c & 127) == 0 && !(fabsf(mean) + fabsf(scale) * app.level_b < kF16Max)) raise_status(ROLAQ_STATUS_RANGE);
+        }
+        const __nv_bfloat16* qb = app.q + ((size_t)b * heads + h) * ROLAQ_D_C;
+        float sp = __bfloat162float(qb[c]) * x_new;
+        if (c < ROLAQ_D_R)
+            sp = fmaf(__bfloat162float(app.qr[((size_t)b * heads + h) * ROLAQ_D_R + c]),
+                      __bfloat162float(app.k_r[(size_t)b * ROLAQ_D_R + c]), sp);
+        s_new = merge_block_sum(sp, s_red) * app.scale_log2;
+        if (h == 0) {
+            // the token's record, as the write path stores it
+            if (c < ROLAQ_CODE_BYTES / 4) s_codes[c] = 0u;
+            __syncthreads();
+            atomicOr(&s_codes[c >> 4], code << (2 * (c & 15)));
+            __syncthreads();
+            long long pid = -1;
+            if (pos / ROLAQ_PAGE_TOKENS < app.max_pages) {
+                pid = app.page_table[(long long)b * app.max_pages + pos / ROLAQ_PAGE_TOKENS];
+                if (pid >= app.num_pages) pid = -1;
+            }
+            if (pid < 0) {
+                if (c == 0) raise_status(ROLAQ_STATUS_BAD_SLOT);
+            } else {
+                uint8_t* page = app.pages + pid * (long long)ROLAQ_PAGE_BYTES;
+                const int row = pos % ROLAQ_PAGE_TOKENS;
+                if (c < ROLAQ_CODE_BYTES / 4)
+                    reinterpret_cast<uint32_t*>(page + ROLAQ_PAGE_CODES_OFFSET + row * ROLAQ_CODE_BYTES)[c] = s_codes[c];
+                if ((c & 127) == 0)
+                    *reinterpret_cast<float2*>(page + ROLAQ_PAGE_META_OFFSET + row * ROLAQ_META_BYTES + 8 * g) =
+                        make_float2(mean, scale);
+                if (c < ROLAQ_KR_BYTES / 8)
+                    reinterpret_cast<uint2*>(page + ROLAQ_PAGE_KR_OFFSET + row * ROLAQ_KR_BYTES)[c] =
+                        reinterpret_cast<const uint2*>(app.k_r + (size_t)b * ROLAQ_D_R)[c];
+                if (prot) {
+                    const int nslot = app.n_sink + app.n_recent;
+                    const int slot = pos < app.n_sink ? pos : app.n_sink + pos % app.n_recent;
+                    app.prot[((size_t)b * nslot + slot) * ROLAQ_D_C + c] = __float2bfloat16_rn(y);
+                }
+            }
+        }
     }
     __syncthreads();
     const int p0 = s_plan[0], np = s_plan[1];
@@ -737,7 +907,7 @@ rolaq_decode_merge(const float* __restrict__ ws_o, const float2* __restrict__ ws
     if (lane == 0) s_red[warp] = M;
     __syncthreads();
     if (threadIdx.x == 0) {
-        float m = -INFINITY;
+        float m = s_new;
         for (int w = 0; w < kWarps; ++w) m = fmaxf(m, s_red[w]);
         s_M = m;
     }
@@ -766,17 +936,18 @@ rolaq_decode_merge(const float* __restrict__ ws_o, const float2* __restrict__ ws
     for (int j = 0; j < 4; ++j) reinterpret_cast<float4*>(s_acc[warp])[lane + 32 * j] = acc[j];
     if (lane == 0) s_red[warp] = den;
     __syncthreads();
+    const float w_new = s_new > -INFINITY ? exp2f(s_new - M) : 0.f;
     if (threadIdx.x == 0) {
         float dsum = 0.f;
         for (int w = 0; w < kWarps; ++w) dsum += s_red[w];
-        s_den = dsum;
+        s_den = dsum + w_new;
     }
     __syncthreads();
     den = s_den;
-    const int c = threadIdx.x;               // one output channel per thread
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) v += s_acc[w][c];
+    v = fmaf(w_new, x_new, v);
     out[((size_t)b * heads + h) * ROLAQ_D_C + c] = den > 0.f ? v / den : 0.f;
     if (lse && threadIdx.x == 0)
         lse[(size_t)b * heads + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;

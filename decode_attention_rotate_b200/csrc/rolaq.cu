@@ -100,6 +100,9 @@ size_t decode_ws_bytes_for(int batch, int heads, int target) {
 
 size_t decode_ws_bytes(int batch, int heads) { return decode_ws_bytes_for(batch, heads, decode_target_items()); }
 
+// Fused append: the new tokens' rotated coordinates, fp32 [batch][512].
+size_t decode_append_ws_bytes(int batch) { return (size_t)batch * ROLAQ_D_C * sizeof(float); }
+
 // Raise a kernel's dynamic shared-memory limit once per device.
 template <typename Kernel>
 void set_smem_limit_once(Kernel k, size_t smem, bool* done) {
@@ -261,18 +264,31 @@ static int decode_check(const rolaq_cache* cache, const rolaq_layer_params* p, c
     return ROLAQ_OK;
 }
 
+// The new tokens of a fused append: rotation planes, latents, RoPE keys (all null: none).
+struct NewTokens {
+    const void* R_split;
+    const void* c;
+    const void* k_r;
+};
+
 // The decode with an explicit split-K target (work items before the per-request
-// remainders); the workspace must hold (target + batch) items.
+// remainders); the workspace must hold (target + batch) items, plus batch x 512 floats
+// of rotated new-token coordinates with a fused append.
 static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* p,
                             const void* q_c_rot_dev, const void* q_R_dev,
                             const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
                             float* out_dev, float* lse_dev,
-                            void* workspace_dev, size_t workspace_bytes, void* stream, int target) {
+                            void* workspace_dev, size_t workspace_bytes, void* stream, int target,
+                            const NewTokens& nt = NewTokens{nullptr, nullptr, nullptr}) {
     int rc = decode_check(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale, out_dev, lse_dev);
     if (rc) return rc;
+    const bool append = nt.R_split != nullptr;
+    if (append && (!nt.c || !nt.k_r || !aligned(nt.R_split, 16) || !aligned(nt.c, 16) || !aligned(nt.k_r, 16)))
+        return ROLAQ_EINVAL;
     if (!workspace_dev || !aligned(workspace_dev, 16)) return ROLAQ_EINVAL;
     if (target < 1) return ROLAQ_ENOSPACE;
-    if (workspace_bytes < decode_ws_bytes_for(batch, heads, target)) return ROLAQ_ENOSPACE;
+    const size_t ws_items = decode_ws_bytes_for(batch, heads, target);
+    if (workspace_bytes < ws_items + (append ? decode_append_ws_bytes(batch) : 0)) return ROLAQ_ENOSPACE;
 
     // The pool as rows of 128 B; one box is a whole page (144 rows).
     CUtensorMap map_page;
@@ -301,6 +317,27 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
     a.ws_o = reinterpret_cast<float*>(workspace_dev);
     a.ws_ml = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(workspace_dev) +
                                         (size_t)items_cap * heads * ROLAQ_D_C * sizeof(float));
+    a.append = append ? 1 : 0;
+    a.app_R = reinterpret_cast<const __nv_bfloat16*>(nt.R_split);
+    a.app_c = reinterpret_cast<const __nv_bfloat16*>(nt.c);
+    a.ws_y = append ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace_dev) + ws_items) : nullptr;
+    AppendArgs ap;
+    ap.y = a.ws_y;
+    ap.k_r = reinterpret_cast<const __nv_bfloat16*>(nt.k_r);
+    ap.q = a.q;
+    ap.qr = a.qr;
+    ap.scale_log2 = a.scale_log2;
+    ap.tau = p->tau;
+    ap.gain = p->gain;
+    ap.level_a = p->level_a;
+    ap.level_b = p->level_b;
+    ap.pages = reinterpret_cast<uint8_t*>(cache->pages_dev);
+    ap.page_table = cache->page_table_dev;
+    ap.num_pages = cache->num_pages;
+    ap.max_pages = cache->max_pages_per_seq;
+    ap.prot = (cache->n_sink + cache->n_recent > 0) ? reinterpret_cast<__nv_bfloat16*>(cache->prot_dev) : nullptr;
+    ap.n_sink = cache->n_sink;
+    ap.n_recent = cache->n_recent;
 
     cudaStream_t s = (cudaStream_t)stream;
     if (heads % 32 == 0) {
@@ -318,7 +355,7 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
     }
     if ((rc = launch_status())) return rc;
     rolaq_decode_merge<<<dim3(batch, heads), kMergeThreads, 0, s>>>(a.ws_o, a.ws_ml, seq_lens_dev, batch, heads,
-                                                         target, out_dev, lse_dev);
+                                                                   target, out_dev, lse_dev, ap);
     return launch_status();
 }
 
@@ -329,6 +366,23 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
                       void* workspace_dev, size_t workspace_bytes, void* stream) {
     return decode_attn_impl(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale, out_dev,
                             lse_dev, workspace_dev, workspace_bytes, stream, decode_target_items());
+}
+
+size_t rolaq_decode_append_workspace_bytes(int batch, int heads) {
+    const size_t base = rolaq_decode_workspace_bytes(batch, heads);
+    return base ? base + decode_append_ws_bytes(batch) : 0;
+}
+
+int rolaq_decode_attn_append(const rolaq_cache* cache, const rolaq_layer_params* p,
+                             const void* R_split_dev, const void* c_new_dev, const void* k_R_new_dev,
+                             const void* q_c_rot_dev, const void* q_R_dev,
+                             const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
+                             float* out_dev, float* lse_dev,
+                             void* workspace_dev, size_t workspace_bytes, void* stream) {
+    if (!R_split_dev || !c_new_dev || !k_R_new_dev) return ROLAQ_EINVAL;
+    return decode_attn_impl(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale, out_dev,
+                            lse_dev, workspace_dev, workspace_bytes, stream, decode_target_items(),
+                            NewTokens{R_split_dev, c_new_dev, k_R_new_dev});
 }
 
 // ---- decode with library-owned scratch -------------------------------------------

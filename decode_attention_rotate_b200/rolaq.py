@@ -20,6 +20,10 @@ D_C = 512
 D_R = 64
 D_NOPE = 128            # per-head no-RoPE query width
 D_V = 128               # per-head value width
+GROUP = 128              # coordinates per quantization group
+GROUPS = 4
+CODE_BYTES = 128         # 512 x 2 bit per token
+META_BYTES = 32          # 4 groups x (mean, scale) fp32
 PAGE_TOKENS = 64
 PAGE_BYTES = 18432
 TOKEN_BYTES = 288
@@ -99,6 +103,11 @@ def lib() -> ctypes.CDLL:
         L.rolaq_decode_attn.restype = i32
         L.rolaq_decode_attn.argtypes = [P(rolaq_cache), P(rolaq_layer_params), vp, vp, vp, i32, i32,
                                         ctypes.c_float, vp, vp, vp, sz, vp]
+        L.rolaq_decode_append_workspace_bytes.restype = sz
+        L.rolaq_decode_append_workspace_bytes.argtypes = [i32, i32]
+        L.rolaq_decode_attn_append.restype = i32
+        L.rolaq_decode_attn_append.argtypes = [P(rolaq_cache), P(rolaq_layer_params), vp, vp, vp, vp, vp, vp,
+                                               i32, i32, ctypes.c_float, vp, vp, vp, sz, vp]
         L.rolaq_decode_attn_static.restype = i32
         L.rolaq_decode_attn_static.argtypes = [P(rolaq_cache), P(rolaq_layer_params), vp, vp, vp, i32, i32,
                                                ctypes.c_float, vp, vp, vp]
@@ -245,6 +254,39 @@ def decode_attn(cache: PagedCache, params: rolaq_layer_params, q_c_rot: torch.Te
     _check("rolaq_decode_attn", lib().rolaq_decode_attn(
         ctypes.byref(d), ctypes.byref(params), _ptr(q_c_rot), _ptr(q_r), _ptr(seq_lens), B, H,
         float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def decode_append_workspace_bytes(batch: int, heads: int) -> int:
+    """rolaq_decode_append_workspace_bytes: scratch rolaq_decode_attn_append needs."""
+    return int(lib().rolaq_decode_append_workspace_bytes(batch, heads))
+
+
+def decode_attn_append(cache: PagedCache, params: rolaq_layer_params, R_split: torch.Tensor,
+                       c_new: torch.Tensor, k_r_new: torch.Tensor, q_c_rot: torch.Tensor, q_r: torch.Tensor,
+                       seq_lens: torch.Tensor, sm_scale: float, out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                       stream=None):
+    """rolaq_decode_attn_append: append token seq_lens[r] - 1 of every request r (c_new bf16
+    [B, 512], k_r_new bf16 [B, 64]) and decode over the cache that includes it; returns
+    (out, lse) as decode_attn."""
+    B, H = int(q_c_rot.shape[0]), int(q_c_rot.shape[1])
+    assert q_c_rot.dtype == torch.bfloat16 and q_r.dtype == torch.bfloat16
+    assert c_new.dtype == torch.bfloat16 and k_r_new.dtype == torch.bfloat16
+    assert tuple(c_new.shape) == (B, D_C) and tuple(k_r_new.shape) == (B, D_R)
+    assert c_new.is_contiguous() and k_r_new.is_contiguous()
+    dev = q_c_rot.device
+    if out is None:
+        out = torch.empty((B, H, D_C), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(decode_append_workspace_bytes(B, H), 16), dtype=torch.uint8, device=dev)
+    d = cache.desc()
+    _check("rolaq_decode_attn_append", lib().rolaq_decode_attn_append(
+        ctypes.byref(d), ctypes.byref(params), _ptr(R_split), _ptr(c_new), _ptr(k_r_new), _ptr(q_c_rot),
+        _ptr(q_r), _ptr(seq_lens), B, H, float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
     return out, lse
 
 

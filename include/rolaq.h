@@ -15,6 +15,7 @@
  *           the coupled gain restores unit response.
  *   [S4.1]  §4.1 "Setup": protection keeps the first 4 sink and the most recent tokens
  *           in BF16.
+ *   [S5.4]  §5.4 "Token Protection": sink plus recent-token budgets kept in BF16.
  *   [A.3]   §A.3 "Calibration and Storage": 288 B per unprotected token per layer
  *           (packed codes + group statistics + BF16 RoPE key); protected tokens also
  *           store BF16 content.
@@ -192,6 +193,39 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
                       const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
                       float* out_dev, float* lse_dev,
                       void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace rolaq_decode_attn_append needs: rolaq_decode_workspace_bytes
+ * plus batch x 2,048 (the new tokens' rotated coordinates, fp32 [batch][512]); 0 where
+ * rolaq_decode_workspace_bytes is 0.                                                   */
+size_t rolaq_decode_append_workspace_bytes(int batch, int heads);
+
+/* Serving step with the per-step write fused into the decode [S4.1], [S5.4],
+ * [A.3]: one new token per request is appended (recent tokens stay protected in bf16,
+ * older ones live as 2-bit codes) and the decode runs over the cache that includes it,
+ * in the two launches of one decode call.  For request r with L = seq_lens_dev[r] >= 1
+ * (the length AFTER the append) the token at position L - 1 is written as
+ * rolaq_quantize_append with req = r, pos = L - 1 and these seq_lens writes it (codes,
+ * statistics, k_R, and its side-store row when protected), from row r of c_new_dev
+ * (bf16 [batch][512]) and k_R_new_dev (bf16 [batch][64]); R_split_dev is the operand of
+ * rolaq_prepare_rotation.  out and lse are those of rolaq_decode_attn over the L tokens:
+ * the new token enters with the value the decode reads from the cache (bf16 y when
+ * protected, else the fp16 mean + scale * level) and a score summed in fp32.  A request
+ * with L <= 0 gets nothing written, out = 0 and lse = -inf.  workspace_dev (16-B
+ * aligned) must hold rolaq_decode_append_workspace_bytes(batch, heads) bytes and needs
+ * no initialisation.  Errors as rolaq_decode_attn; a null or misaligned (16 B)
+ * R_split_dev, c_new_dev or k_R_new_dev gives ROLAQ_EINVAL.  A position whose page is
+ * not mapped in page_table sets ROLAQ_STATUS_BAD_SLOT and is not stored; the decode
+ * still counts the token.  How the work is spread: in the split kernel one otherwise
+ * idle warp of every CTA computes a few coordinates of y = c . R for all new tokens (so
+ * R is read once, spread over the SMs); the merge kernel, which runs after it, finishes
+ * the write and adds the new token's term.  Calls that overlap on the GPU must not share
+ * a workspace or append to the same request.                                            */
+int rolaq_decode_attn_append(const rolaq_cache* cache, const rolaq_layer_params* p,
+                             const void* R_split_dev, const void* c_new_dev, const void* k_R_new_dev,
+                             const void* q_c_rot_dev, const void* q_R_dev,
+                             const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
+                             float* out_dev, float* lse_dev,
+                             void* workspace_dev, size_t workspace_bytes, void* stream);
 
 /* Decode without a caller-provided workspace.  Same arguments, result and errors as
  * rolaq_decode_attn, except that the split-K scratch lives in a fixed array inside the

@@ -164,3 +164,26 @@ def test_static_decode_rejects_before_any_launch(lib):
     c = _cache(batch=5000)
     assert lib.rolaq_decode_attn_static(ctypes.byref(c), ctypes.byref(p), ptr, ptr, ptr, 5000, 16,
                                         0.07, None, ptr, None) == -1
+
+
+def test_append_decode_rejects_before_any_launch(lib):
+    """The fused append + decode checks its extra pointers and its larger workspace on the
+    host, after the decode's own checks, before any CUDA call."""
+    p = R.rolaq_layer_params(0.9, 1.0, 0.45, 1.5)
+    ptr = 1 << 22
+    need = lib.rolaq_decode_append_workspace_bytes(2, 16)
+    assert need == lib.rolaq_decode_workspace_bytes(2, 16) + 2 * 512 * 4
+    assert lib.rolaq_decode_append_workspace_bytes(2, 24) == 0
+    assert lib.rolaq_decode_append_workspace_bytes(0, 16) == 0
+
+    def call(Rs=ptr, c=ptr, k=ptr, ws=ptr, nbytes=need, batch=2, heads=16, cache=None):
+        cd = cache if cache is not None else _cache(batch=2)
+        return lib.rolaq_decode_attn_append(ctypes.byref(cd), ctypes.byref(p), Rs, c, k, ptr, ptr, ptr, batch,
+                                            heads, 0.07, ptr, ptr, ws, nbytes, None)
+    assert call(Rs=None) == -1 and call(c=None) == -1 and call(k=None) == -1
+    assert call(c=ptr + 2) == -1 and call(k=ptr + 8) == -1 and call(Rs=ptr + 4) == -1
+    assert call(heads=24) == -4
+    assert call(batch=3) == -1                                  # beyond the cache's batch
+    assert call(ws=None) == -1
+    # enough for the plain decode but not for the new tokens' coordinates
+    assert call(nbytes=lib.rolaq_decode_workspace_bytes(2, 16)) == -2

@@ -57,6 +57,12 @@ def test_static_scratch_rejects_oversized_requests():
     assert need > R.STATIC_SCRATCH_BYTES
     big_q = torch.zeros((1000, 128, 512), dtype=torch.bfloat16, device=DEV)
     big_r = torch.zeros((1000, 128, 64), dtype=torch.bfloat16, device=DEV)
+    # a batch beyond the cache's is an argument error, checked first
     with pytest.raises(R.RolaqError) as e:
         R.decode_attn_static(cache, p, big_q, big_r, lens, SM_SCALE)
+    assert e.value.code == -1
+    # a cache of 1000 requests (all on one page; nothing is launched): no room for the plan
+    wide = R.PagedCache(cache.num_pages, torch.zeros((1000, 1), dtype=torch.int32), device=DEV, pages=cache.pages)
+    with pytest.raises(R.RolaqError) as e:
+        R.decode_attn_static(wide, p, big_q, big_r, lens, SM_SCALE)
     assert e.value.code == -2
