@@ -55,6 +55,7 @@ constexpr int kSCol = 0;                            // TMEM: S tiles at columns 
 constexpr int kOCol = 64;                           //       O at 64.. (HC per group)
 constexpr int kXqCol = 256;                         //       token-major x (QK's A): 256..511
 template <int HC> __host__ __device__ constexpr int tmem_cols_for() { return 512; }
+constexpr int kPBufs = 3;                           // probability buffers (PV's B operand)
 constexpr float kRescaleLog2 = 8.f;
 constexpr float kF16Max = 65504.f;
 
@@ -102,11 +103,10 @@ struct DecodeSmem {
     alignas(1024) uint8_t stage[kStages][ROLAQ_PAGE_BYTES];
     alignas(128) uint8_t qc[HC * ROLAQ_D_C * 2];          // fp16 query, QK B operand
     alignas(128) uint8_t qr[HC * ROLAQ_D_R * 2];          // bf16 RoPE query, B operand
-    alignas(128) uint8_t P[2][HC * kPageTok * 2];         // fp16 probabilities, PV B operand
+    alignas(128) uint8_t P[kPBufs][HC * kPageTok * 2];    // fp16 probabilities, PV B operand
     float red[4][HC];                                     // softmax warps: per-warp head values
     float mref[HC];                                       // running reference max per head
     float alpha[HC];                                      // its last rescale factor
-    int vote[2][4];
     alignas(8) uint64_t full[kStages];     // page copy landed
     alignas(8) uint64_t pfree[kStages];    // page read by the dequant warps and the QK MMAs
     alignas(8) uint64_t xready[2][2];      // x tile half written (channel groups 0-1 / 2-3)
@@ -115,7 +115,8 @@ struct DecodeSmem {
     alignas(8) uint64_t xq_free;           // QK of the page done with the token-major x
     alignas(8) uint64_t sfull[2];          // QK of the tile done
     alignas(8) uint64_t sfree[2];          // scores read by the softmax warps
-    alignas(8) uint64_t pready[2];         // P written (and O rescaled if needed)
+    alignas(8) uint64_t pready[kPBufs];    // P written (and O rescaled if needed)
+    alignas(8) uint64_t pdone[kPBufs];     // PV done with the P buffer
     int valid[kStages];
     uint32_t tmem_base;
     int plan[4];
@@ -442,7 +443,10 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             }
             mbar_init(smem_u32(&sm.sfull[s]), 1);
             mbar_init(smem_u32(&sm.sfree[s]), 4);
+        }
+        for (int s = 0; s < kPBufs; ++s) {
             mbar_init(smem_u32(&sm.pready[s]), 4);
+            mbar_init(smem_u32(&sm.pdone[s]), 1);
         }
         for (int hf = 0; hf < 2; ++hf) mbar_init(smem_u32(&sm.xq_full[hf]), (kDecodeThreads / 32 - kDqWarp0) / 2);
         mbar_init(smem_u32(&sm.xq_free), 1);
@@ -556,13 +560,13 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
             const uint64_t dxm = smem_desc(smem_u32(sm.x[0]), kXAtom, 1024, 2);
             const uint64_t dp = smem_desc(smem_u32(sm.P[0]), 128, 1024, 0);
             auto pv = [&](int j) {
-                const int bj = j & 1;
-                mbar_wait(smem_u32(&sm.pready[bj]), (unsigned)((j >> 1) & 1), &sm.abort);
+                const int bj = j & 1, pj = j % kPBufs;
+                mbar_wait(smem_u32(&sm.pready[pj]), (unsigned)((j / kPBufs) & 1), &sm.abort);
                 mbar_wait(smem_u32(&sm.xready[bj][0]), (unsigned)((j >> 1) & 1), &sm.abort);
                 mbar_wait(smem_u32(&sm.xready[bj][1]), (unsigned)((j >> 1) & 1), &sm.abort);
                 __syncwarp();
                 tc_fence_after();
-                const uint64_t da = dxm + (uint64_t)(bj * (kXTile >> 4)), db = dp + (uint64_t)(bj * (sizeof(sm.P[0]) >> 4));
+                const uint64_t da = dxm + (uint64_t)(bj * (kXTile >> 4)), db = dp + (uint64_t)(pj * (sizeof(sm.P[0]) >> 4));
                 const uint32_t first = j > 0 ? 1u : 0u;
                 if (elect_one()) {
 #pragma unroll
@@ -574,6 +578,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                         if (g == 1) umma_commit(smem_u32(&sm.xfree[bj][0]));   // groups 0-1 read
                     }
                     umma_commit(smem_u32(&sm.xfree[bj][1]));
+                    umma_commit(smem_u32(&sm.pdone[pj]));
                 }
                 __syncwarp();
             };
@@ -673,10 +678,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                 }
             }
             // the four softmax warps agree on whether any head's reference moves
-            const bool wup = __any_sync(0xffffffffu, up);
-            if (lane == 0) sm.vote[bi][q] = wup ? 1 : 0;
-            named_bar_sync(1, 128);
-            const bool any = (sm.vote[bi][0] | sm.vote[bi][1] | sm.vote[bi][2] | sm.vote[bi][3]) != 0;
+            const bool any = named_bar_or(1, 128, up);
             if (any) {
                 // per-head max over the tile: lanes sharing i4 hold the same heads
 #pragma unroll
@@ -731,9 +733,10 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                 }
                 named_bar_sync(1, 128);        // red / alpha are read by every softmax warp before reuse
             }
-            // P buffer bi is free once PV(i - 2) has completed
-            if (i >= 2) mbar_wait(smem_u32(&sm.xfree[bi][1]), (unsigned)(((i - 2) >> 1) & 1), &sm.abort);
-            uint8_t* P = sm.P[bi];
+            // P buffer i % kPBufs is free once PV(i - kPBufs) has completed
+            const int pi = i % kPBufs;
+            if (i >= kPBufs) mbar_wait(smem_u32(&sm.pdone[pi]), (unsigned)((i / kPBufs - 1) & 1), &sm.abort);
+            uint8_t* P = sm.P[pi];
 #pragma unroll
             for (int e = 0; e < kE; ++e)
 #pragma unroll
@@ -744,7 +747,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
                 }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.pready[bi]));
+            if (lane == 0) mbar_arrive(smem_u32(&sm.pready[pi]));
         }
         // ---- this item's partial: O (rows = slots), per-head (m, l) ----------------
         if (T > 0) mbar_wait(smem_u32(&sm.xfree[(T - 1) & 1][1]), (unsigned)(((T - 1) >> 1) & 1), &sm.abort);
