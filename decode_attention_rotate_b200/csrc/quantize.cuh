@@ -24,12 +24,12 @@ namespace rolaq {
 
 constexpr int kQTileM = 128;                  // tokens per tile (TMEM lanes)
 constexpr int kQN = ROLAQ_GROUP;              // output coordinates per job: one group
-constexpr int kQK = 32;                       // K per chunk (64-byte rows, 64B swizzle)
-constexpr int kQKSteps = ROLAQ_D_C / kQK;     // 16
-constexpr int kQStages = 5;
+constexpr int kQK = 64;                       // K per chunk (128-byte rows, 128B swizzle)
+constexpr int kQKSteps = ROLAQ_D_C / kQK;     // 8
+constexpr int kQStages = 3;
 constexpr int kQThreads = 320;
 constexpr int kQPlanes = 3;
-constexpr uint32_t kQChunkBytes = kQTileM * kQK * 2;      // 8 KB (c chunk or one R-plane chunk)
+constexpr uint32_t kQChunkBytes = kQTileM * kQK * 2;      // 16 KB (c chunk or one R-plane chunk)
 
 struct QuantArgs {
     uint8_t* pages;
@@ -47,7 +47,7 @@ struct QuantArgs {
 };
 
 struct QuantSmem {
-    alignas(1024) uint8_t a[kQKSteps][kQChunkBytes];        // resident c tile, 16 K chunks
+    alignas(1024) uint8_t a[kQKSteps][kQChunkBytes];        // resident c tile, 8 K chunks
     alignas(1024) uint8_t b[kQStages][2][kQChunkBytes];     // streamed R-plane chunks
     alignas(8) uint64_t a_full[kQKSteps];
     uint64_t a_free[kQKSteps];
@@ -59,11 +59,12 @@ struct QuantSmem {
     int abort;
 };
 
-// Shared-memory matrix descriptor: K-major operand, 64-byte rows with 64B swizzle,
-// 8-row core groups 512 bytes apart.
-__device__ __forceinline__ uint64_t umma_desc_sw64(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (32ull << 32) | (1ull << 46) |
-           (4ull << 61);
+static_assert(sizeof(QuantSmem) + 1024 <= 227 * 1024, "write-path shared memory");
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte rows with 128B swizzle,
+// 8-row core groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+    return smem_desc(saddr, 16, 1024, 2);
 }
 // Instruction descriptor: bf16 x bf16 -> f32, both K-major, M = 128, N = 128.
 constexpr uint32_t kQIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kQN >> 3) << 17) |
@@ -89,14 +90,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
           "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
         : "r"(taddr));
 }
-// 32 columns of y = chain A + chain B (fp32 add of the two K-half accumulators).
+// 32 columns of y = chain A + chain B (fp32 add of the two K-half accumulators), chain B
+// read 16 columns at a time to keep the register peak low.
 __device__ __forceinline__ void load_y32(uint32_t col_a, uint32_t col_b, float (&y)[32]) {
-    float t[32];
     tmem_ld32(col_a, y);
-    tmem_ld32(col_b, t);
-    tmem_ld_wait();
 #pragma unroll
-    for (int j = 0; j < 32; ++j) y[j] += t[j];
+    for (int h = 0; h < 2; ++h) {
+        uint32_t t[16];
+        tmem_ld16(col_b + 16 * h, t);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) y[16 * h + j] += __uint_as_float(t[j]);
+    }
 }
 
 // Quantize one 128-coordinate group of one token straight from TMEM (this thread's lane;
@@ -268,12 +273,12 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
                             const uint32_t sb0 = smem_u32(sm.b[st][0]), sb1 = smem_u32(sm.b[st][1]);
                             if (elect_one()) {
 #pragma unroll
-                                for (int k16 = 0; k16 < 2; ++k16) {
-                                    const uint64_t da = umma_desc_sw64(sa + 32 * k16);
-                                    const uint64_t db0 = umma_desc_sw64(sb0 + 32 * k16);
+                                for (int k16 = 0; k16 < kQK / 16; ++k16) {
+                                    const uint64_t da = umma_desc_sw128(sa + 32 * k16);
+                                    const uint64_t db0 = umma_desc_sw128(sb0 + 32 * k16);
                                     if (pass == 0) {
                                         umma_bf16(d_a, da, db0, (kc | k16) != 0);
-                                        umma_bf16(d_a, da, umma_desc_sw64(sb1 + 32 * k16), 1u);
+                                        umma_bf16(d_a, da, umma_desc_sw128(sb1 + 32 * k16), 1u);
                                     } else if (kc < kQKSteps / 2) {
                                         umma_bf16(d_a, da, db0, 1u);
                                     } else {

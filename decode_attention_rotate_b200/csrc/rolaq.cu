@@ -211,9 +211,9 @@ int rolaq_quantize_append(const rolaq_cache* cache, const rolaq_layer_params* p,
 
     CUtensorMap map_c, map_r;
     if (!encode_2d(&map_c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(c_dev), ROLAQ_D_C,
-                   (uint64_t)n, ROLAQ_D_C * 2, kQK, kQTileM, CU_TENSOR_MAP_SWIZZLE_64B) ||
+                   (uint64_t)n, ROLAQ_D_C * 2, kQK, kQTileM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&map_r, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, const_cast<void*>(R_split_dev), ROLAQ_D_C,
-                   kQPlanes * ROLAQ_D_C, ROLAQ_D_C * 2, kQK, kQN, CU_TENSOR_MAP_SWIZZLE_64B))
+                   kQPlanes * ROLAQ_D_C, ROLAQ_D_C * 2, kQK, kQN, CU_TENSOR_MAP_SWIZZLE_128B))
         return ROLAQ_ECUDA;
 
     QuantArgs a;
