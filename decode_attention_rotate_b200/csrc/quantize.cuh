@@ -5,9 +5,10 @@
 //
 // rolaq_quantize_kernel is persistent (one CTA per SM).  A tile is 128 tokens (the TMEM
 // lanes); its c block stays in shared memory while the four groups of 128 output
-// coordinates are produced one after the other (one job per group).  Warp roles:
-//   warp 8      producer: bulk tensor copies of the c tile (16 chunks of 128 x 32) and
-//               of the R-plane chunks (128 x 32) each job needs;
+// coordinates are produced one after the other (one job per group); the tiles of a last,
+// at most half-full round are split in two units of two groups.  Warp roles:
+//   warp 8      producer: bulk tensor copies of the c tile (8 chunks of 128 x 64) and
+//               of the R-plane chunks (128 x 64, 128-byte swizzle) each job needs;
 //   warp 9      allocates 512 TMEM columns and issues tcgen05.mma (M=128, N=128, K=16,
 //               bf16 in, fp32 accumulate).  R = R_hi + R_mid + R_lo (three bf16 planes,
 //               ~2^-26 relative).  The tensor cores truncate each fp32 accumulation step
@@ -90,43 +91,39 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
           "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
         : "r"(taddr));
 }
-// 32 columns of y = chain A + chain B (fp32 add of the two K-half accumulators), chain B
-// read 16 columns at a time to keep the register peak low.
-__device__ __forceinline__ void load_y32(uint32_t col_a, uint32_t col_b, float (&y)[32]) {
-    tmem_ld32(col_a, y);
+// 16 columns of y = chain A + chain B (fp32 add of the two K-half accumulators).
+__device__ __forceinline__ void load_y16(uint32_t col_a, uint32_t col_b, float (&y)[16]) {
+    uint32_t ua[16], ub[16];
+    tmem_ld16(col_a, ua);
+    tmem_ld16(col_b, ub);
+    tmem_ld_wait();
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        uint32_t t[16];
-        tmem_ld16(col_b + 16 * h, t);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) y[16 * h + j] += __uint_as_float(t[j]);
-    }
+    for (int j = 0; j < 16; ++j) y[j] = __uint_as_float(ua[j]) + __uint_as_float(ub[j]);
 }
 
 // Quantize one 128-coordinate group of one token straight from TMEM (this thread's lane;
-// chain A at col_a.., chain B at col_b..), streaming 32 columns at a time in three
+// chain A at col_a.., chain B at col_b..), streaming 16 columns at a time in three
 // passes: mean, population std, then codes (and the bf16 copy for a protected token).
 // All lanes of the warp must call it (the TMEM loads are warp-wide); `store` is false for
 // lanes without a valid target.
 __device__ __forceinline__ void quantize_group_tmem(uint32_t col_a, uint32_t col_b, float tau, float gain,
                                                     bool store, uint8_t* dst_codes, float* dst_meta,
                                                     __nv_bfloat16* dst_prot) {
-    float y[32];
+    float y[16];
     float s = 0.f;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-        load_y32(col_a + 32 * c, col_b + 32 * c, y);
+    for (int c = 0; c < 8; ++c) {
+        load_y16(col_a + 16 * c, col_b + 16 * c, y);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) s += y[j];
+        for (int j = 0; j < 16; ++j) s += y[j];
     }
     const float mean = s * (1.f / 128.f);
     float ss = 0.f;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-        load_y32(col_a + 32 * c, col_b + 32 * c, y);
+    for (int c = 0; c < 8; ++c) {
+        load_y16(col_a + 16 * c, col_b + 16 * c, y);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 16; ++j) {
             const float d = y[j] - mean;
             ss = fmaf(d, d, ss);
         }
@@ -134,35 +131,43 @@ __device__ __forceinline__ void quantize_group_tmem(uint32_t col_a, uint32_t col
     const float sd = sqrtf(ss * (1.f / 128.f));
     // z = (y - mean) / sd against -tau, 0, tau; a group with sd == 0 gets z = 0.
     const float inv = sd > 0.f ? 1.f / sd : 0.f;
-    uint32_t w[8];
+#pragma unroll 1
+    for (int c = 0; c < 8; ++c) {
+        load_y16(col_a + 16 * c, col_b + 16 * c, y);
+        uint32_t acc = 0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        load_y32(col_a + 32 * c, col_b + 32 * c, y);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            uint32_t acc = 0;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float z = (y[16 * h + j] - mean) * inv;
-                const uint32_t code = (uint32_t)(z >= -tau) + (uint32_t)(z >= 0.f) + (uint32_t)(z >= tau);
-                acc |= code << (2 * j);
-            }
-            w[2 * c + h] = acc;
+        for (int j = 0; j < 16; ++j) {
+            const float z = (y[j] - mean) * inv;
+            const uint32_t code = (uint32_t)(z >= -tau) + (uint32_t)(z >= 0.f) + (uint32_t)(z >= tau);
+            acc |= code << (2 * j);
         }
+        if (store) reinterpret_cast<uint32_t*>(dst_codes)[c] = acc;      // 16 codes
         if (store && dst_prot) {
-            uint4* dp = reinterpret_cast<uint4*>(dst_prot + 32 * c);
+            uint4* dp = reinterpret_cast<uint4*>(dst_prot + 16 * c);
 #pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8)
+            for (int q8 = 0; q8 < 2; ++q8)
                 dp[q8] = make_uint4(pack_bf16(y[8 * q8 + 0], y[8 * q8 + 1]), pack_bf16(y[8 * q8 + 2], y[8 * q8 + 3]),
                                     pack_bf16(y[8 * q8 + 4], y[8 * q8 + 5]), pack_bf16(y[8 * q8 + 6], y[8 * q8 + 7]));
         }
     }
-    if (store) {
-        uint4* dc = reinterpret_cast<uint4*>(dst_codes);
-        dc[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dc[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        *reinterpret_cast<float2*>(dst_meta) = make_float2(mean, gain * sd);
-    }
+    if (store) *reinterpret_cast<float2*>(dst_meta) = make_float2(mean, gain * sd);
+}
+
+// Work units of the persistent grid: CTA b takes tiles b, b + grid, ... whole (all four
+// groups); when the last round is at most half full, each of its tiles is split in two
+// units of two groups (groups 0-1 and 2-3 on CTAs 2j and 2j + 1), so that round costs
+// half a tile.  Every role of a CTA walks the same units.
+struct QUnit { int tile, g0, ng; };
+__device__ __forceinline__ int q_unit_count(int n_tiles, int cta) {
+    const int grid = (int)gridDim.x, full = n_tiles / grid, rem = n_tiles % grid;
+    const bool split = rem > 0 && 2 * rem <= grid;
+    return full + ((split ? cta < 2 * rem : cta < rem) ? 1 : 0);
+}
+__device__ __forceinline__ QUnit q_unit(int n_tiles, int cta, int k) {
+    const int grid = (int)gridDim.x, full = n_tiles / grid, rem = n_tiles % grid;
+    if (k < full) return QUnit{k * grid + cta, 0, ROLAQ_GROUPS};
+    if (rem > 0 && 2 * rem <= grid) return QUnit{full * grid + cta / 2, 2 * (cta & 1), 2};
+    return QUnit{full * grid + cta, 0, ROLAQ_GROUPS};
 }
 
 __global__ void __launch_bounds__(kQThreads, 1)
@@ -210,11 +215,14 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
             uint32_t it = 0;
             int tl = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tl)
-                for (int g = 0; g < ROLAQ_GROUPS && ok; ++g)
+            const int nu = q_unit_count(n_tiles, (int)blockIdx.x);
+            for (int un = 0; un < nu && ok; ++un, ++tl) {
+                const QUnit w = q_unit(n_tiles, (int)blockIdx.x, un);
+                const int tile = w.tile;
+                for (int g = w.g0; g < w.g0 + w.ng && ok; ++g)
                     for (int pass = 0; pass < 2 && ok; ++pass)
                         for (int kc = 0; kc < kQKSteps; ++kc, ++it) {
-                            if (g == 0 && pass == 0) {
+                            if (g == w.g0 && pass == 0) {
                                 if (tl > 0 && !mbar_wait(smem_u32(&sm.a_free[kc]), (tl - 1) & 1, &sm.abort)) {
                                     ok = false;
                                     break;
@@ -240,6 +248,7 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
                                 tma_load_2d(smem_u32(sm.b[st][0]), &map_r, kc * kQK, n0, fb);
                             }
                         }
+            }
         }
     } else if (warp == 9) {
         // ----------------------------------------------------------------- MMA ----
@@ -252,8 +261,10 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
             uint32_t it = 0, job = 0;
             int tl = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x, ++tl)
-                for (int g = 0; g < ROLAQ_GROUPS && ok; ++g, ++job) {
+            const int nu = q_unit_count(n_tiles, (int)blockIdx.x);
+            for (int un = 0; un < nu && ok; ++un, ++tl) {
+                const QUnit w = q_unit(n_tiles, (int)blockIdx.x, un);
+                for (int g = w.g0; g < w.g0 + w.ng && ok; ++g, ++job) {
                     const uint32_t buf = job & 1, use = job >> 1;
                     if (use >= 1)
                         ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.tempty[buf]), (use - 1) & 1, &sm.abort));
@@ -262,7 +273,7 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
                     const uint32_t d_a = tmem + buf * 2 * kQN, d_b = d_a + kQN;
                     for (int pass = 0; pass < 2 && ok; ++pass)
                         for (int kc = 0; kc < kQKSteps; ++kc, ++it) {
-                            if (g == 0 && pass == 0)
+                            if (g == w.g0 && pass == 0)
                                 ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.a_full[kc]), tl & 1, &sm.abort));
                             const int st = it % kQStages;
                             if (ok)
@@ -286,7 +297,7 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
                                     }
                                 }
                                 umma_commit(smem_u32(&sm.empty[st]));
-                                if (g == ROLAQ_GROUPS - 1 && pass == 1) umma_commit(smem_u32(&sm.a_free[kc]));
+                                if (g == w.g0 + w.ng - 1 && pass == 1) umma_commit(smem_u32(&sm.a_free[kc]));
                             }
                             __syncwarp();
                         }
@@ -295,6 +306,7 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
                         __syncwarp();
                     }
                 }
+            }
         }
     } else {
         // ------------------------------------------------------------ epilogue ----
@@ -303,10 +315,12 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
         const int q = warp & 3, set = warp >> 2;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         uint32_t use = 0;
-        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        const int nu = q_unit_count(n_tiles, (int)blockIdx.x);
+        for (int un = 0; un < nu; ++un) {
+            const QUnit w = q_unit(n_tiles, (int)blockIdx.x, un);
             // Target slot of this thread's token, looked up before the accumulator is ready
             // so the dependent global loads overlap the MMAs.
-            const int tok = tile * kQTileM + 32 * q + lane;
+            const int tok = w.tile * kQTileM + 32 * q + lane;
             long long pid = -1;
             int rq = -1, ps = 0;
             if (tok < args.n) {
@@ -329,13 +343,13 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
                 else if (args.n_recent > 0 && ps >= args.seq_lens[rq] - args.n_recent)
                     prot_row = (long long)rq * nslot + args.n_sink + ps % args.n_recent;
             }
-            if (store && set == 0) {
+            if (store && set == 0 && w.g0 == 0) {
                 const uint4* src = reinterpret_cast<const uint4*>(args.k_r + (size_t)tok * ROLAQ_D_R);
                 uint4* dst = reinterpret_cast<uint4*>(page + ROLAQ_PAGE_KR_OFFSET + row * ROLAQ_KR_BYTES);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) dst[j] = src[j];
             }
-            for (int g = set; g < ROLAQ_GROUPS; g += 2, ++use) {
+            for (int g = w.g0 + set; g < w.g0 + w.ng; g += 2, ++use) {
                 const bool got = mbar_wait(smem_u32(&sm.tfull[set]), use & 1, &sm.abort);
                 tc_fence_after();
                 __nv_bfloat16* prot = prot_row >= 0 ? args.prot + prot_row * ROLAQ_D_C + 128 * g : nullptr;

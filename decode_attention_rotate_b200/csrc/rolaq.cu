@@ -236,8 +236,10 @@ int rolaq_quantize_append(const rolaq_cache* cache, const rolaq_layer_params* p,
     const size_t smem = sizeof(QuantSmem) + 1024;
     static bool attr_done[kMaxDevices] = {false};
     set_smem_limit_once(rolaq_quantize_kernel, smem, attr_done);
+    // one CTA per SM, or two per tile for calls of fewer tiles than half the SMs (the
+    // kernel then splits every tile's groups between a pair of CTAs)
     const int tiles = (n + kQTileM - 1) / kQTileM;
-    const int grid = tiles < current_sms() ? tiles : current_sms();
+    const int grid = 2 * tiles < current_sms() ? 2 * tiles : current_sms();
     rolaq_quantize_kernel<<<grid, kQThreads, smem, (cudaStream_t)stream>>>(map_c, map_r, a);
     return launch_status();
 }
