@@ -622,37 +622,50 @@ def bench_bf16_baseline(args, dev, world, w, dec_ms):
 
 
 def bench_all_protected(args, dev, dec_ms):
-    """This library's decode with quantization disabled: every token protected (its bf16
-    latent read from the side store, 1,152 B per token with the RoPE key), the same
-    4 x 262,144 tokens at 16 heads as the bench."""
+    """This library's decode with quantization disabled: every token protected, its bf16
+    latent read from the side store (1,152 B per token with the RoPE key), the same
+    4 x 262,144 tokens at 16 heads as the bench; through the BF16 decode
+    (rolaq_decode_attn_bf16), and for comparison through the 2-bit-page decode, which
+    still stages each token's page."""
     w = W.Workload("all_protected_4x256k_h16", 4, (262144,) * 4, 16, n_sink=0, n_recent=262144, seed=1010)
+    hbm, _, src = peaks()
     try:
         lay = DecodeLayer(w, 0, dev)
         lay.fill(w, 0, dev)
         ws = torch.empty(R.decode_workspace_bytes(w.batch, w.heads), dtype=torch.uint8, device=dev)
         lens = torch.as_tensor(w.seq_lens, dtype=torch.int32, device=dev)
-        call = lambda: R.decode_attn(lay.cache, lay.params, lay.q_c, lay.q_r, lens, SM_SCALE, lay.out, lay.lse, ws)
-        for _ in range(max(args.warmup, 3)):
-            call()
-        torch.cuda.synchronize()
-        assert R.get_status() == 0
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 10
-        t0.record()
-        for _ in range(reps):
-            call()
-        t1.record()
-        torch.cuda.synchronize()
-        ms = t0.elapsed_time(t1) / reps
+
+        def timed(fn):
+            for _ in range(max(args.warmup, 3)):
+                fn()
+            torch.cuda.synchronize()
+            assert R.get_status() == 0
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 10
+            t0.record()
+            for _ in range(reps):
+                fn()
+            t1.record()
+            torch.cuda.synchronize()
+            return t0.elapsed_time(t1) / reps
+        ms = timed(lambda: R.decode_attn_bf16(lay.cache, lay.params, lay.q_c, lay.q_r, lens, SM_SCALE, lay.out,
+                                              lay.lse, ws))
+        ms2 = timed(lambda: R.decode_attn(lay.cache, lay.params, lay.q_c, lay.q_r, lens, SM_SCALE, lay.out,
+                                          lay.lse, ws))
     except Exception as e:                      # report, never lose the bench line
         return {"unavailable": f"{type(e).__name__}: {e}"[:200]}
     finally:
         torch.cuda.empty_cache()
     nbytes = w.total_tokens * R.BF16_TOKEN_BYTES
-    return {"kernel": "rolaq_decode_split + merge, every token protected (bf16 side store)",
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"kernel": "rolaq_decode_bf16 + merge (BF16 decode: side-store rows and RoPE rows by bulk tensor copies)",
             "workload": "4 x 262144 tokens, 16 heads, one layer", "bytes_per_token": R.BF16_TOKEN_BYTES,
-            "ms_per_call": round(ms, 4), "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
-            "time_ratio_over_2bit": round(ms / dec_ms, 3)}
+            "ms_per_call": round(ms, 4), "GB_s": round(gbs, 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                         "frac": round(gbs / hbm, 4), "peak_source": src},
+            "time_ratio_over_2bit": round(ms / dec_ms, 3),
+            "via_2bit_page_decode": {"ms_per_call": round(ms2, 4),
+                                     "GB_s": round(nbytes / (ms2 * 1e-3) / 1e9, 1)}}
 
 
 # ------------------------------------------------------------ profiling cases ----

@@ -409,6 +409,164 @@ __device__ __forceinline__ void append_rotate(const DecodeArgs& args, int cta, i
     }
 }
 
+// Softmax role (warps 4..7) of the decode kernels: scores from tensor memory, the lazy
+// reference max, P into shared memory (fp16, or bf16 when the x operand is bf16), O
+// rescaled in place when the reference moves, and at the end the item's partial (O rows
+// in slot order for the 2-bit kernel, in channel order for the bf16 one, and (m, l) per
+// head).  pv_wait(j) returns once the PV of page j has completed.
+template <bool kBf16P> __device__ __forceinline__ uint16_t p_bits(float p);
+template <> __device__ __forceinline__ uint16_t p_bits<false>(float p) { return __half_as_ushort(__float2half_rn(p)); }
+template <> __device__ __forceinline__ uint16_t p_bits<true>(float p) { return __bfloat16_as_ushort(__float2bfloat16_rn(p)); }
+
+template <int HC, bool kBf16P, bool kSlotOrder, typename Smem, typename PvWait>
+__device__ __forceinline__ void softmax_role(Smem& sm, const DecodeArgs& args, uint32_t tmem, int warp, int lane,
+                                             int b, int first_page, int T, int Lkv, int h0, PvWait pv_wait) {
+    // ------------------------------------------------------------- softmax ----
+    // Warp q reads TMEM lane quarter q: S rows 16q..16q+15 (M = 64) in lanes 0..15 with
+    // the 16x256b shape, so lane (r, i) holds rows 16q + r and 16q + r + 8 of heads
+    // 8k + 2i and 8k + 2i + 1 (k < HC / 8); O rows (slots) 32q..32q+31 of every group.
+    constexpr int kE = HC / 4;             // heads per thread
+    const int q = warp - kSoftWarp0;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const int r = lane >> 2, i4 = lane & 3;
+    const int rows[2] = {16 * q + r, 16 * q + r + 8};
+    int heads[kE];
+#pragma unroll
+    for (int e = 0; e < kE; ++e) heads[e] = 8 * (e >> 1) + 2 * i4 + (e & 1);
+    float m_ref[kE], l[kE];
+#pragma unroll
+    for (int e = 0; e < kE; ++e) { m_ref[e] = -INFINITY; l[e] = 0.f; }
+    long long pid_next = page_id(args, b, first_page);
+    for (int i = 0; i < T; ++i) {
+        const int bi = i & 1;
+        const bool vpage = page_ok(args, pid_next);
+        if (i + 1 < T) pid_next = page_id(args, b, first_page + i + 1);
+        mbar_wait(smem_u32(&sm.sfull[bi]), (unsigned)((i >> 1) & 1), &sm.abort);
+        __syncwarp();
+        tc_fence_after();
+        uint32_t u[HC / 2];
+        tmem_ld_scores(tmem + lane_base + kSCol + HC * bi, u);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.sfree[bi]));
+        // s[e][j]: head heads[e], row rows[j]
+        float s2[kE][2];
+        bool up = false;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const bool valid = vpage && (first_page + i) * kPageTok + rows[j] < Lkv;
+#pragma unroll
+            for (int e = 0; e < kE; ++e) {
+                const uint32_t raw = u[(e >> 1) * 4 + 2 * j + (e & 1)];
+                s2[e][j] = valid ? __uint_as_float(raw) * args.scale_log2 : -INFINITY;
+                up |= s2[e][j] > m_ref[e] + kRescaleLog2 || (m_ref[e] == -INFINITY && s2[e][j] > -INFINITY);
+            }
+        }
+        // the four softmax warps agree on whether any head's reference moves
+        const bool any = named_bar_or(1, 128, up);
+        if (any) {
+            // per-head max over the tile: lanes sharing i4 hold the same heads
+#pragma unroll
+            for (int e = 0; e < kE; ++e) {
+                float mx = fmaxf(s2[e][0], s2[e][1]);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                if (r == 0) sm.red[q][heads[e]] = mx;
+            }
+            named_bar_sync(1, 128);
+            if (q == 0 && lane < HC) {
+                // one thread per head: new reference and factor for all warps
+                const int h = lane;
+                const float tm = fmaxf(fmaxf(sm.red[0][h], sm.red[1][h]), fmaxf(sm.red[2][h], sm.red[3][h]));
+                const float mo = sm.mref[h];
+                float al = 1.f, mn = mo;
+                if (tm > mo + kRescaleLog2 || (mo == -INFINITY && tm > -INFINITY)) {
+                    al = (mo == -INFINITY) ? 0.f : ex2(mo - tm);
+                    mn = tm;
+                }
+                sm.alpha[h] = al;
+                sm.mref[h] = mn;
+            }
+            named_bar_sync(1, 128);
+            bool moved = false;
+#pragma unroll
+            for (int e = 0; e < kE; ++e) {
+                const float al = sm.alpha[heads[e]];
+                m_ref[e] = sm.mref[heads[e]];
+                l[e] *= al;
+            }
+#pragma unroll
+            for (int h = 0; h < HC; ++h) moved |= sm.alpha[h] != 1.f;
+            if (moved && i > 0) {
+                // O holds PV of tiles 0..i-1: wait for PV(i-1), scale this quarter's lanes
+                pv_wait(i - 1);
+                __syncwarp();
+                tc_fence_after();
+#pragma unroll 1
+                for (int gc = 0; gc < 4 * (HC / 16); ++gc) {       // 16-column slices of O
+                    uint32_t v[16];
+                    tmem_ld16(tmem + lane_base + kOCol + 16 * gc, v);
+                    tmem_ld_wait();
+                    const int hb = 16 * (gc % (HC / 16));            // first head of the slice
+#pragma unroll
+                    for (int h = 0; h < 16; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * sm.alpha[hb + h]);
+                    tmem_st16(tmem + lane_base + kOCol + 16 * gc, v);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+            }
+            named_bar_sync(1, 128);        // red / alpha are read by every softmax warp before reuse
+        }
+        // P buffer i % kPBufs is free once PV(i - kPBufs) has completed
+        const int pi = i % kPBufs;
+        if (i >= kPBufs) mbar_wait(smem_u32(&sm.pdone[pi]), (unsigned)((i / kPBufs - 1) & 1), &sm.abort);
+        uint8_t* P = sm.P[pi];
+#pragma unroll
+        for (int e = 0; e < kE; ++e)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const float p = (m_ref[e] == -INFINITY) ? 0.f : ex2(s2[e][j] - m_ref[e]);
+                l[e] += p;
+                *reinterpret_cast<uint16_t*>(P + plain_off(heads[e], rows[j], 8 * 128)) = p_bits<kBf16P>(p);
+            }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.pready[pi]));
+    }
+    // ---- this item's partial: O (rows = slots), per-head (m, l) ----------------
+    if (T > 0) pv_wait(T - 1);
+    __syncwarp();
+    tc_fence_after();
+    const int m = 32 * q + lane;           // O row = slot (or channel) within the group
+#pragma unroll 1
+    for (int gc = 0; gc < 4 * (HC / 16); ++gc) {           // 16-column slices of O
+        const int g = gc / (HC / 16), hb = 16 * (gc % (HC / 16));
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_base + kOCol + 16 * gc, v);
+        tmem_ld_wait();
+        float* dst = args.ws_o + ((size_t)blockIdx.x * args.heads + h0 + hb) * ROLAQ_D_C + 128 * g + (kSlotOrder ? slot_channel(m) : m);
+#pragma unroll
+        for (int h = 0; h < 16; ++h) dst[(size_t)h * ROLAQ_D_C] = __uint_as_float(v[h]);
+    }
+    // row sums: lanes sharing i4 (8 per warp) and the four warps
+#pragma unroll
+    for (int e = 0; e < kE; ++e) {
+        float v = l[e];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        if (r == 0) sm.red[q][heads[e]] = v;
+    }
+    named_bar_sync(1, 128);
+    if (q == 0 && lane < HC) {
+        const int h = lane;
+        args.ws_ml[(size_t)blockIdx.x * args.heads + h0 + h] =
+            make_float2(sm.mref[h], (sm.red[0][h] + sm.red[1][h]) + (sm.red[2][h] + sm.red[3][h]));
+    }
+}
+
 template <int HC>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
 rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArgs args) {
@@ -636,149 +794,9 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
         if (appender) append_rotate(args, (int)blockIdx.x, (int)gridDim.x);
     } else if (warp >= kSoftWarp0) {
         // ------------------------------------------------------------- softmax ----
-        // Warp q reads TMEM lane quarter q: S rows 16q..16q+15 (M = 64) in lanes 0..15 with
-        // the 16x256b shape, so lane (r, i) holds rows 16q + r and 16q + r + 8 of heads
-        // 8k + 2i and 8k + 2i + 1 (k < HC / 8); O rows (slots) 32q..32q+31 of every group.
-        constexpr int kE = HC / 4;             // heads per thread
-        const int q = warp - kSoftWarp0;
-        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const int r = lane >> 2, i4 = lane & 3;
-        const int rows[2] = {16 * q + r, 16 * q + r + 8};
-        int heads[kE];
-#pragma unroll
-        for (int e = 0; e < kE; ++e) heads[e] = 8 * (e >> 1) + 2 * i4 + (e & 1);
-        float m_ref[kE], l[kE];
-#pragma unroll
-        for (int e = 0; e < kE; ++e) { m_ref[e] = -INFINITY; l[e] = 0.f; }
-        long long pid_next = page_id(args, b, page_of(0));
-        for (int i = 0; i < T; ++i) {
-            const int bi = i & 1;
-            const bool vpage = page_ok(args, pid_next);
-            if (i + 1 < T) pid_next = page_id(args, b, page_of(i + 1));
-            mbar_wait(smem_u32(&sm.sfull[bi]), (unsigned)((i >> 1) & 1), &sm.abort);
-            __syncwarp();
-            tc_fence_after();
-            uint32_t u[HC / 2];
-            tmem_ld_scores(tmem + lane_base + kSCol + HC * bi, u);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.sfree[bi]));
-            // s[e][j]: head heads[e], row rows[j]
-            float s2[kE][2];
-            bool up = false;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const bool valid = vpage && page_of(i) * kPageTok + rows[j] < Lkv;
-#pragma unroll
-                for (int e = 0; e < kE; ++e) {
-                    const uint32_t raw = u[(e >> 1) * 4 + 2 * j + (e & 1)];
-                    s2[e][j] = valid ? __uint_as_float(raw) * args.scale_log2 : -INFINITY;
-                    up |= s2[e][j] > m_ref[e] + kRescaleLog2 || (m_ref[e] == -INFINITY && s2[e][j] > -INFINITY);
-                }
-            }
-            // the four softmax warps agree on whether any head's reference moves
-            const bool any = named_bar_or(1, 128, up);
-            if (any) {
-                // per-head max over the tile: lanes sharing i4 hold the same heads
-#pragma unroll
-                for (int e = 0; e < kE; ++e) {
-                    float mx = fmaxf(s2[e][0], s2[e][1]);
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                    if (r == 0) sm.red[q][heads[e]] = mx;
-                }
-                named_bar_sync(1, 128);
-                if (q == 0 && lane < HC) {
-                    // one thread per head: new reference and factor for all warps
-                    const int h = lane;
-                    const float tm = fmaxf(fmaxf(sm.red[0][h], sm.red[1][h]), fmaxf(sm.red[2][h], sm.red[3][h]));
-                    const float mo = sm.mref[h];
-                    float al = 1.f, mn = mo;
-                    if (tm > mo + kRescaleLog2 || (mo == -INFINITY && tm > -INFINITY)) {
-                        al = (mo == -INFINITY) ? 0.f : ex2(mo - tm);
-                        mn = tm;
-                    }
-                    sm.alpha[h] = al;
-                    sm.mref[h] = mn;
-                }
-                named_bar_sync(1, 128);
-                bool moved = false;
-#pragma unroll
-                for (int e = 0; e < kE; ++e) {
-                    const float al = sm.alpha[heads[e]];
-                    m_ref[e] = sm.mref[heads[e]];
-                    l[e] *= al;
-                }
-#pragma unroll
-                for (int h = 0; h < HC; ++h) moved |= sm.alpha[h] != 1.f;
-                if (moved && i > 0) {
-                    // O holds PV of tiles 0..i-1: wait for PV(i-1), scale this quarter's lanes
-                    mbar_wait(smem_u32(&sm.xfree[(i - 1) & 1][1]), (unsigned)(((i - 1) >> 1) & 1), &sm.abort);
-                    __syncwarp();
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int gc = 0; gc < 4 * (HC / 16); ++gc) {       // 16-column slices of O
-                        uint32_t v[16];
-                        tmem_ld16(tmem + lane_base + kOCol + 16 * gc, v);
-                        tmem_ld_wait();
-                        const int hb = 16 * (gc % (HC / 16));            // first head of the slice
-#pragma unroll
-                        for (int h = 0; h < 16; ++h) v[h] = __float_as_uint(__uint_as_float(v[h]) * sm.alpha[hb + h]);
-                        tmem_st16(tmem + lane_base + kOCol + 16 * gc, v);
-                    }
-                    tmem_st_wait();
-                    tc_fence_before();
-                }
-                named_bar_sync(1, 128);        // red / alpha are read by every softmax warp before reuse
-            }
-            // P buffer i % kPBufs is free once PV(i - kPBufs) has completed
-            const int pi = i % kPBufs;
-            if (i >= kPBufs) mbar_wait(smem_u32(&sm.pdone[pi]), (unsigned)((i / kPBufs - 1) & 1), &sm.abort);
-            uint8_t* P = sm.P[pi];
-#pragma unroll
-            for (int e = 0; e < kE; ++e)
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const float p = (m_ref[e] == -INFINITY) ? 0.f : ex2(s2[e][j] - m_ref[e]);
-                    l[e] += p;
-                    *reinterpret_cast<__half*>(P + plain_off(heads[e], rows[j], 8 * 128)) = __float2half_rn(p);
-                }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&sm.pready[pi]));
-        }
-        // ---- this item's partial: O (rows = slots), per-head (m, l) ----------------
-        if (T > 0) mbar_wait(smem_u32(&sm.xfree[(T - 1) & 1][1]), (unsigned)(((T - 1) >> 1) & 1), &sm.abort);
-        __syncwarp();
-        tc_fence_after();
-        const int m = 32 * q + lane;           // O row = slot within the group
-#pragma unroll 1
-        for (int gc = 0; gc < 4 * (HC / 16); ++gc) {           // 16-column slices of O
-            const int g = gc / (HC / 16), hb = 16 * (gc % (HC / 16));
-            uint32_t v[16];
-            tmem_ld16(tmem + lane_base + kOCol + 16 * gc, v);
-            tmem_ld_wait();
-            float* dst = args.ws_o + ((size_t)blockIdx.x * args.heads + h0 + hb) * ROLAQ_D_C + 128 * g + slot_channel(m);
-#pragma unroll
-            for (int h = 0; h < 16; ++h) dst[(size_t)h * ROLAQ_D_C] = __uint_as_float(v[h]);
-        }
-        // row sums: lanes sharing i4 (8 per warp) and the four warps
-#pragma unroll
-        for (int e = 0; e < kE; ++e) {
-            float v = l[e];
-            v += __shfl_xor_sync(0xffffffffu, v, 4);
-            v += __shfl_xor_sync(0xffffffffu, v, 8);
-            v += __shfl_xor_sync(0xffffffffu, v, 16);
-            if (r == 0) sm.red[q][heads[e]] = v;
-        }
-        named_bar_sync(1, 128);
-        if (q == 0 && lane < HC) {
-            const int h = lane;
-            args.ws_ml[(size_t)blockIdx.x * args.heads + h0 + h] =
-                make_float2(sm.mref[h], (sm.red[0][h] + sm.red[1][h]) + (sm.red[2][h] + sm.red[3][h]));
-        }
+        softmax_role<HC, false, true>(sm, args, tmem, warp, lane, b, first_page, T, Lkv, h0, [&](int j) {
+            mbar_wait(smem_u32(&sm.xfree[j & 1][1]), (unsigned)((j >> 1) & 1), &sm.abort);
+        });
     }
     tc_fence_before();
     __syncthreads();

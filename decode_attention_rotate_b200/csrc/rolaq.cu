@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_bf16.cuh"
 #include "project.cuh"
 #include "quantize.cuh"
 
@@ -281,9 +282,12 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
                             const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
                             float* out_dev, float* lse_dev,
                             void* workspace_dev, size_t workspace_bytes, void* stream, int target,
-                            const NewTokens& nt = NewTokens{nullptr, nullptr, nullptr}) {
+                            const NewTokens& nt = NewTokens{nullptr, nullptr, nullptr}, bool bf16 = false) {
     int rc = decode_check(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale, out_dev, lse_dev);
     if (rc) return rc;
+    const int nslot = cache->n_sink + cache->n_recent;
+    if (bf16 && (!cache->prot_dev || nslot <= 0)) return ROLAQ_EINVAL;
+    if (bf16 && (cache->n_sink % ROLAQ_PAGE_TOKENS || cache->n_recent % ROLAQ_PAGE_TOKENS)) return ROLAQ_EUNSUPPORTED;
     const bool append = nt.R_split != nullptr;
     if (append && (!nt.c || !nt.k_r || !aligned(nt.R_split, 16) || !aligned(nt.c, 16) || !aligned(nt.k_r, 16)))
         return ROLAQ_EINVAL;
@@ -342,7 +346,27 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
     ap.n_recent = cache->n_recent;
 
     cudaStream_t s = (cudaStream_t)stream;
-    if (heads % 32 == 0) {
+    if (bf16) {
+        // the side store as rows of 512 bf16 (boxes of 64 x 64, 128-byte swizzle) and the
+        // pool as rows of 128 B (boxes of the 64 RoPE rows of a page)
+        CUtensorMap map_x, map_kr;
+        if (!encode_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cache->prot_dev, ROLAQ_D_C,
+                       (uint64_t)cache->batch * nslot, ROLAQ_D_C * 2, 64, ROLAQ_PAGE_TOKENS, CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !encode_2d(&map_kr, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache->pages_dev, 128, rows, 128, 128,
+                       ROLAQ_PAGE_TOKENS, CU_TENSOR_MAP_SWIZZLE_128B))
+            return ROLAQ_ECUDA;
+        if (heads % 32 == 0) {
+            const size_t smem = sizeof(Bf16Smem<32>) + 1024;
+            static bool attr_done[kMaxDevices] = {false};
+            set_smem_limit_once(rolaq_decode_bf16<32>, smem, attr_done);
+            rolaq_decode_bf16<32><<<dim3(items_cap, heads / 32), kBf16Threads, smem, s>>>(map_x, map_kr, a);
+        } else {
+            const size_t smem = sizeof(Bf16Smem<16>) + 1024;
+            static bool attr_done[kMaxDevices] = {false};
+            set_smem_limit_once(rolaq_decode_bf16<16>, smem, attr_done);
+            rolaq_decode_bf16<16><<<dim3(items_cap, heads / 16), kBf16Threads, smem, s>>>(map_x, map_kr, a);
+        }
+    } else if (heads % 32 == 0) {
         // 32 heads per CTA (twice the work per tensor-core instruction and per
         // dequantised tile)
         const size_t smem = sizeof(DecodeSmem<32>) + 1024;
@@ -368,6 +392,16 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
                       void* workspace_dev, size_t workspace_bytes, void* stream) {
     return decode_attn_impl(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale, out_dev,
                             lse_dev, workspace_dev, workspace_bytes, stream, decode_target_items());
+}
+
+int rolaq_decode_attn_bf16(const rolaq_cache* cache, const rolaq_layer_params* p,
+                           const void* q_c_rot_dev, const void* q_R_dev,
+                           const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
+                           float* out_dev, float* lse_dev,
+                           void* workspace_dev, size_t workspace_bytes, void* stream) {
+    return decode_attn_impl(cache, p, q_c_rot_dev, q_R_dev, seq_lens_dev, batch, heads, sm_scale, out_dev,
+                            lse_dev, workspace_dev, workspace_bytes, stream, decode_target_items(),
+                            NewTokens{nullptr, nullptr, nullptr}, true);
 }
 
 size_t rolaq_decode_append_workspace_bytes(int batch, int heads) {

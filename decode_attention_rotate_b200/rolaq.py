@@ -103,6 +103,9 @@ def lib() -> ctypes.CDLL:
         L.rolaq_decode_attn.restype = i32
         L.rolaq_decode_attn.argtypes = [P(rolaq_cache), P(rolaq_layer_params), vp, vp, vp, i32, i32,
                                         ctypes.c_float, vp, vp, vp, sz, vp]
+        L.rolaq_decode_attn_bf16.restype = i32
+        L.rolaq_decode_attn_bf16.argtypes = [P(rolaq_cache), P(rolaq_layer_params), vp, vp, vp, i32, i32,
+                                             ctypes.c_float, vp, vp, vp, sz, vp]
         L.rolaq_decode_append_workspace_bytes.restype = sz
         L.rolaq_decode_append_workspace_bytes.argtypes = [i32, i32]
         L.rolaq_decode_attn_append.restype = i32
@@ -252,6 +255,28 @@ def decode_attn(cache: PagedCache, params: rolaq_layer_params, q_c_rot: torch.Te
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
     d = cache.desc()
     _check("rolaq_decode_attn", lib().rolaq_decode_attn(
+        ctypes.byref(d), ctypes.byref(params), _ptr(q_c_rot), _ptr(q_r), _ptr(seq_lens), B, H,
+        float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def decode_attn_bf16(cache: PagedCache, params: rolaq_layer_params, q_c_rot: torch.Tensor, q_r: torch.Tensor,
+                     seq_lens: torch.Tensor, sm_scale: float, out: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                     stream=None):
+    """rolaq_decode_attn_bf16: decode from the bf16 side store (every token protected);
+    arguments and result as decode_attn."""
+    B, H = int(q_c_rot.shape[0]), int(q_c_rot.shape[1])
+    assert q_c_rot.dtype == torch.bfloat16 and q_r.dtype == torch.bfloat16
+    dev = q_c_rot.device
+    if out is None:
+        out = torch.empty((B, H, D_C), dtype=torch.float32, device=dev)
+    if lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(decode_workspace_bytes(B, H), 16), dtype=torch.uint8, device=dev)
+    d = cache.desc()
+    _check("rolaq_decode_attn_bf16", lib().rolaq_decode_attn_bf16(
         ctypes.byref(d), ctypes.byref(params), _ptr(q_c_rot), _ptr(q_r), _ptr(seq_lens), B, H,
         float(sm_scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out, lse

@@ -92,7 +92,8 @@ extern "C" {
 
 /* Device status bits reported by rolaq_get_status(). */
 #define ROLAQ_STATUS_BAD_PAGE   1  /* page-table entry < 0 or >= num_pages (skipped)  */
-#define ROLAQ_STATUS_BAD_SLOT   2  /* append target outside its request's pages       */
+#define ROLAQ_STATUS_BAD_SLOT   2  /* append target outside its request's pages, or (BF16
+                                      decode) a position without a bf16 copy          */
 #define ROLAQ_STATUS_TIMEOUT    4  /* a pipeline wait gave up (results of that call invalid) */
 #define ROLAQ_STATUS_RANGE      8  /* a decoded x or a query element beyond the fp16 range
                                       (|x|, |q| >= 65504): that decode result is invalid  */
@@ -193,6 +194,24 @@ int rolaq_decode_attn(const rolaq_cache* cache, const rolaq_layer_params* p,
                       const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
                       float* out_dev, float* lse_dev,
                       void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/* BF16 decode on the same cache [S4.1], [A.3]: quantisation disabled, every token read
+ * from its bf16 copy in the side store (the content the protected tokens keep) with its
+ * RoPE key from the page; the 2-bit codes are not read.  Result as rolaq_decode_attn for
+ * a cache whose every token is protected; arguments, workspace and errors as
+ * rolaq_decode_attn, and in addition: the cache must have a side store (else
+ * ROLAQ_EINVAL) with n_sink and n_recent multiples of 64 (else ROLAQ_EUNSUPPORTED), so
+ * that each 64-token page maps to one run of side-store rows.  A request with
+ * L > n_sink + n_recent has positions without a bf16 copy: ROLAQ_STATUS_BAD_SLOT is set
+ * and its result is not valid.  Arithmetic: x, q_c_rot and the probabilities enter the
+ * tensor-core products as bf16 (both operands of one product share a type), sums fp32.
+ * Each page is moved with bulk tensor copies (64 side-store rows as eight 64 x 64 boxes
+ * with the 128-byte swizzle, plus the page's 64 RoPE rows): 1,152 B per token.          */
+int rolaq_decode_attn_bf16(const rolaq_cache* cache, const rolaq_layer_params* p,
+                           const void* q_c_rot_dev, const void* q_R_dev,
+                           const int32_t* seq_lens_dev, int batch, int heads, float sm_scale,
+                           float* out_dev, float* lse_dev,
+                           void* workspace_dev, size_t workspace_bytes, void* stream);
 
 /* Bytes of device workspace rolaq_decode_attn_append needs: rolaq_decode_workspace_bytes
  * plus batch x 2,048 (the new tokens' rotated coordinates, fp32 [batch][512]); 0 where

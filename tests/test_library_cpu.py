@@ -187,3 +187,23 @@ def test_append_decode_rejects_before_any_launch(lib):
     assert call(ws=None) == -1
     # enough for the plain decode but not for the new tokens' coordinates
     assert call(nbytes=lib.rolaq_decode_workspace_bytes(2, 16)) == -2
+
+
+def test_bf16_decode_rejects_before_any_launch(lib):
+    """The BF16 decode needs a side store whose windows are multiples of 64 tokens."""
+    p = R.rolaq_layer_params(0.9, 1.0, 0.45, 1.5)
+    ptr = 1 << 22
+    need = lib.rolaq_decode_workspace_bytes(2, 16)
+
+    def call(**kw):
+        c = _cache(batch=2, **kw)
+        return lib.rolaq_decode_attn_bf16(ctypes.byref(c), ctypes.byref(p), ptr, ptr, ptr, 2, 16, 0.07, ptr, ptr,
+                                          ptr, need, None)
+    assert call() == -1                                      # no side store
+    assert call(prot=ptr, n_sink=4, n_recent=128) == -4      # sink window not a multiple of 64
+    assert call(prot=ptr, n_sink=0, n_recent=100) == -4
+    c = _cache(batch=2, prot=ptr, n_recent=128)
+    assert lib.rolaq_decode_attn_bf16(ctypes.byref(c), ctypes.byref(p), ptr, ptr, ptr, 2, 24, 0.07, ptr, ptr,
+                                      ptr, need, None) == -4     # heads not a multiple of 16
+    assert lib.rolaq_decode_attn_bf16(ctypes.byref(c), ctypes.byref(p), ptr, ptr, ptr, 2, 16, 0.07, ptr, ptr,
+                                      ptr, need - 16, None) == -2
