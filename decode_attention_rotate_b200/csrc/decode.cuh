@@ -653,6 +653,7 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     auto page_of = [&](int k) { return first_page + k; };
+    if (threadIdx.x == 0) grid_launch_dependents();     // the merge may be scheduled as CTAs finish
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer ----
@@ -853,6 +854,9 @@ rolaq_decode_merge(const float* __restrict__ ws_o, const float2* __restrict__ ws
     const int b = blockIdx.x, h = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kWarps = kMergeThreads / 32;
+    // launched as a programmatic dependent of the split kernel: everything below reads
+    // its output, so wait for it (a no-op for an ordinary launch)
+    grid_dependency_wait();
     const int c = threadIdx.x;               // one channel per thread
     if (warp == 0) {
         PlanInfo pi = plan_lookup(seq_lens, batch, target, -1, b, app.y != nullptr ? 1 : 0);

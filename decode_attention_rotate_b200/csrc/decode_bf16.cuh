@@ -127,6 +127,7 @@ rolaq_decode_bf16(const __grid_constant__ CUtensorMap map_x, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int nslot = args.n_sink + args.n_recent;
+    if (threadIdx.x == 0) grid_launch_dependents();     // the merge may be scheduled as CTAs finish
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer ----

@@ -380,8 +380,21 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
         rolaq_decode_split<16><<<dim3(items_cap, heads / 16), kDecodeThreads, smem, s>>>(map_page, a);
     }
     if ((rc = launch_status())) return rc;
-    rolaq_decode_merge<<<dim3(batch, heads), kMergeThreads, 0, s>>>(a.ws_o, a.ws_ml, seq_lens_dev, batch, heads,
-                                                                   target, out_dev, lse_dev, ap);
+    // the merge as a programmatic dependent of the split kernel (it waits for the split's
+    // completion itself), so that its launch overlaps the split's last CTAs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(batch, heads);
+    cfg.blockDim = dim3(kMergeThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, rolaq_decode_merge, (const float*)a.ws_o, (const float2*)a.ws_ml, seq_lens_dev,
+                           batch, heads, target, out_dev, lse_dev, ap) != cudaSuccess)
+        return ROLAQ_ECUDA;
     return launch_status();
 }
 
