@@ -580,6 +580,9 @@ rolaq_decode_split(const __grid_constant__ CUtensorMap map_page, const DecodeArg
         *reinterpret_cast<DecodeSmem<HC>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int hc = blockIdx.y;                 // HC-head chunk
+    // launched as a programmatic dependent of the previous kernel in the stream: wait for
+    // it before the first read of any input or write of the workspace
+    grid_dependency_wait();
 
     if (warp == 0) {
         PlanInfo pi = plan_lookup(args.seq_lens, args.batch, args.target_items, (int)blockIdx.x, -1, args.append);
@@ -855,8 +858,10 @@ rolaq_decode_merge(const float* __restrict__ ws_o, const float2* __restrict__ ws
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int kWarps = kMergeThreads / 32;
     // launched as a programmatic dependent of the split kernel: everything below reads
-    // its output, so wait for it (a no-op for an ordinary launch)
+    // its output, so wait for it (a no-op for an ordinary launch); the next kernel may then
+    // be scheduled as merge CTAs finish
     grid_dependency_wait();
+    if (threadIdx.x == 0) grid_launch_dependents();
     const int c = threadIdx.x;               // one channel per thread
     if (warp == 0) {
         PlanInfo pi = plan_lookup(seq_lens, batch, target, -1, b, app.y != nullptr ? 1 : 0);

@@ -68,6 +68,7 @@ rolaq_decode_bf16(const __grid_constant__ CUtensorMap map_x, const __grid_consta
         *reinterpret_cast<Bf16Smem<HC>*>(smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h0 = blockIdx.y * HC;
+    grid_dependency_wait();                    // the previous kernel's output is visible from here
 
     if (warp == 0) {
         PlanInfo pi = plan_lookup(args.seq_lens, args.batch, args.target_items, (int)blockIdx.x, -1, 0);

@@ -267,6 +267,26 @@ static int decode_check(const rolaq_cache* cache, const rolaq_layer_params* p, c
     return ROLAQ_OK;
 }
 
+// Launch as a programmatic dependent of the previous kernel in the stream (the kernel
+// itself waits with griddepcontrol.wait before it touches memory the previous one may use).
+extern "C++" {
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                    Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+}  // extern "C++"
+
 // The new tokens of a fused append: rotation planes, latents, RoPE keys (all null: none).
 struct NewTokens {
     const void* R_split;
@@ -359,12 +379,16 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
             const size_t smem = sizeof(Bf16Smem<32>) + 1024;
             static bool attr_done[kMaxDevices] = {false};
             set_smem_limit_once(rolaq_decode_bf16<32>, smem, attr_done);
-            rolaq_decode_bf16<32><<<dim3(items_cap, heads / 32), kBf16Threads, smem, s>>>(map_x, map_kr, a);
+            if (launch_dependent(rolaq_decode_bf16<32>, dim3(items_cap, heads / 32), dim3(kBf16Threads), smem, s,
+                                 map_x, map_kr, a) != cudaSuccess)
+                return ROLAQ_ECUDA;
         } else {
             const size_t smem = sizeof(Bf16Smem<16>) + 1024;
             static bool attr_done[kMaxDevices] = {false};
             set_smem_limit_once(rolaq_decode_bf16<16>, smem, attr_done);
-            rolaq_decode_bf16<16><<<dim3(items_cap, heads / 16), kBf16Threads, smem, s>>>(map_x, map_kr, a);
+            if (launch_dependent(rolaq_decode_bf16<16>, dim3(items_cap, heads / 16), dim3(kBf16Threads), smem, s,
+                                 map_x, map_kr, a) != cudaSuccess)
+                return ROLAQ_ECUDA;
         }
     } else if (heads % 32 == 0) {
         // 32 heads per CTA (twice the work per tensor-core instruction and per
@@ -372,28 +396,22 @@ static int decode_attn_impl(const rolaq_cache* cache, const rolaq_layer_params* 
         const size_t smem = sizeof(DecodeSmem<32>) + 1024;
         static bool attr_done[kMaxDevices] = {false};
         set_smem_limit_once(rolaq_decode_split<32>, smem, attr_done);
-        rolaq_decode_split<32><<<dim3(items_cap, heads / 32), kDecodeThreads, smem, s>>>(map_page, a);
+        if (launch_dependent(rolaq_decode_split<32>, dim3(items_cap, heads / 32), dim3(kDecodeThreads), smem, s,
+                             map_page, a) != cudaSuccess)
+            return ROLAQ_ECUDA;
     } else {
         const size_t smem = sizeof(DecodeSmem<16>) + 1024;
         static bool attr_done[kMaxDevices] = {false};
         set_smem_limit_once(rolaq_decode_split<16>, smem, attr_done);
-        rolaq_decode_split<16><<<dim3(items_cap, heads / 16), kDecodeThreads, smem, s>>>(map_page, a);
+        if (launch_dependent(rolaq_decode_split<16>, dim3(items_cap, heads / 16), dim3(kDecodeThreads), smem, s,
+                             map_page, a) != cudaSuccess)
+            return ROLAQ_ECUDA;
     }
     if ((rc = launch_status())) return rc;
     // the merge as a programmatic dependent of the split kernel (it waits for the split's
     // completion itself), so that its launch overlaps the split's last CTAs
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(batch, heads);
-    cfg.blockDim = dim3(kMergeThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, rolaq_decode_merge, (const float*)a.ws_o, (const float2*)a.ws_ml, seq_lens_dev,
-                           batch, heads, target, out_dev, lse_dev, ap) != cudaSuccess)
+    if (launch_dependent(rolaq_decode_merge, dim3(batch, heads), dim3(kMergeThreads), 0, s, (const float*)a.ws_o,
+                         (const float2*)a.ws_ml, seq_lens_dev, batch, heads, target, out_dev, lse_dev, ap) != cudaSuccess)
         return ROLAQ_ECUDA;
     return launch_status();
 }
