@@ -120,6 +120,8 @@ rolaq_fold_query_kernel(const __grid_constant__ CUtensorMap map_wq, const __nv_b
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
+    grid_dependency_wait();                    // launched as a dependent: inputs visible from here
+    if (threadIdx.x == 0) grid_launch_dependents();
     if (threadIdx.x == 0) {
         mbar_arrive_expect_tx(smem_u32(&sm.full), 2 * kPjBlock);
         for (int c = 0; c < 2; ++c)
@@ -203,6 +205,8 @@ rolaq_unfold_output_kernel(const __grid_constant__ CUtensorMap map_wo, const flo
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
+    grid_dependency_wait();                    // launched as a dependent: inputs visible from here
+    if (threadIdx.x == 0) grid_launch_dependents();
     if (threadIdx.x == 0) {
         for (int kc = 0; kc < kChunks; ++kc) {
             mbar_arrive_expect_tx(smem_u32(&sm.full[kc]), 2 * kPjBlock);

@@ -206,6 +206,8 @@ rolaq_quantize_kernel(const __grid_constant__ CUtensorMap map_c,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    grid_dependency_wait();                    // launched as a dependent: inputs visible from here
+    if (threadIdx.x == 0) grid_launch_dependents();
 
     if (warp == 8) {
         // ------------------------------------------------------------- producer --

@@ -69,6 +69,26 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, void* base, uint64_t in
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Launch as a programmatic dependent of the previous kernel in the stream (the kernel
+// itself waits with griddepcontrol.wait before it touches memory the previous one may use).
+extern "C++" {
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                    Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+}  // extern "C++"
+
 int check_cache(const rolaq_cache* c) {
     if (!c || !c->pages_dev || !c->page_table_dev || c->num_pages <= 0 || c->batch <= 0 ||
         c->max_pages_per_seq <= 0)
@@ -241,7 +261,9 @@ int rolaq_quantize_append(const rolaq_cache* cache, const rolaq_layer_params* p,
     // kernel then splits every tile's groups between a pair of CTAs)
     const int tiles = (n + kQTileM - 1) / kQTileM;
     const int grid = 2 * tiles < current_sms() ? 2 * tiles : current_sms();
-    rolaq_quantize_kernel<<<grid, kQThreads, smem, (cudaStream_t)stream>>>(map_c, map_r, a);
+    if (launch_dependent(rolaq_quantize_kernel, dim3(grid), dim3(kQThreads), smem, (cudaStream_t)stream, map_c, map_r,
+                         a) != cudaSuccess)
+        return ROLAQ_ECUDA;
     return launch_status();
 }
 
@@ -267,25 +289,6 @@ static int decode_check(const rolaq_cache* cache, const rolaq_layer_params* p, c
     return ROLAQ_OK;
 }
 
-// Launch as a programmatic dependent of the previous kernel in the stream (the kernel
-// itself waits with griddepcontrol.wait before it touches memory the previous one may use).
-extern "C++" {
-template <typename... KArgs, typename... Args>
-inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                                    Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
-}  // extern "C++"
 
 // The new tokens of a fused append: rotation planes, latents, RoPE keys (all null: none).
 struct NewTokens {
@@ -523,8 +526,10 @@ int rolaq_fold_query(const void* q_nope_dev, const void* W_q_dev, int batch, int
     const size_t smem = sizeof(FoldQSmem) + 1024;
     static bool attr_done[kMaxDevices] = {false};
     set_smem_limit_once(rolaq_fold_query_kernel, smem, attr_done);
-    rolaq_fold_query_kernel<<<dim3(ROLAQ_D_C / 128, heads), kPjThreads, smem, (cudaStream_t)stream>>>(
-        map, static_cast<const __nv_bfloat16*>(q_nope_dev), batch, heads, static_cast<__nv_bfloat16*>(q_c_rot_dev));
+    if (launch_dependent(rolaq_fold_query_kernel, dim3(ROLAQ_D_C / 128, heads), dim3(kPjThreads), smem,
+                         (cudaStream_t)stream, map, static_cast<const __nv_bfloat16*>(q_nope_dev), batch, heads,
+                         static_cast<__nv_bfloat16*>(q_c_rot_dev)) != cudaSuccess)
+        return ROLAQ_ECUDA;
     return launch_status();
 }
 
@@ -541,7 +546,9 @@ int rolaq_unfold_output(const float* out_dev, const void* W_o_dev, int batch, in
     const size_t smem = sizeof(UnfoldSmem) + 1024;
     static bool attr_done[kMaxDevices] = {false};
     set_smem_limit_once(rolaq_unfold_output_kernel, smem, attr_done);
-    rolaq_unfold_output_kernel<<<heads, kPjThreads, smem, (cudaStream_t)stream>>>(map, out_dev, batch, heads, v_dev);
+    if (launch_dependent(rolaq_unfold_output_kernel, dim3(heads), dim3(kPjThreads), smem, (cudaStream_t)stream, map,
+                         out_dev, batch, heads, v_dev) != cudaSuccess)
+        return ROLAQ_ECUDA;
     return launch_status();
 }
 
