@@ -11,21 +11,26 @@
 //                     32 heads);
 //   warps 8..15       dequantise: thread (token t, group g) forms the four fp16 values
 //                     mean + scale * level of its (token, group) and turns its 128 codes
-//                     into x with one PRMT per pair, stored straight into a 128-byte-
-//                     swizzled x tile [64 tokens][512 channels] (two tiles, double
-//                     buffered).  fp16, not bf16: channels sharing a code share one
-//                     rounding error, which bf16 makes ~5x too large in the output;
-//   warp 1            issues the tensor-core MMAs (warp-uniform loop, one elected lane
-//                     per batch of instructions): QK as tcgen05.mma M = 64 tokens,
-//                     N = HC heads, K = 512 (fp16, A = the x tile) plus K = 64 (bf16,
-//                     A = the staged page's RoPE rows), S in tensor memory; PV as
-//                     tcgen05.mma M = 128 channels of a group, N = HC heads, K = 64
-//                     tokens, A = the same x tile read transposed (MN-major), B = P,
-//                     O (fp32) accumulated in tensor memory;
-//   warps 4..7        softmax: one tensor-memory load gives a token's HC scores; the
-//                     running max moves only when a score exceeds it by more than 2^8
-//                     (a vote in the common case), in which case O is rescaled before
-//                     the next PV; P goes to shared memory as the fp16 B operand.
+//                     into x with one PRMT per pair (one selector per four codes), then
+//                     writes x twice: token-major into tensor memory (M = 64 layout, QK's
+//                     A operand) and into a 128-byte-swizzled shared-memory tile
+//                     [64 tokens][512 channels] (PV's A operand; two tiles).  fp16, not
+//                     bf16: channels sharing a code share one rounding error, which bf16
+//                     makes ~5x too large in the output;
+//   warp 1            issues QK (warp-uniform loop, one elected lane per batch of
+//                     instructions): tcgen05.mma M = 64 tokens, N = HC heads, K = 512
+//                     (fp16, A = x in tensor memory) plus K = 64 (bf16, A = the staged
+//                     page's RoPE rows), S in tensor memory;
+//   warp 2            issues PV: tcgen05.mma M = 128 channels of a group, N = HC heads,
+//                     K = 64 tokens, A = the shared-memory tile read transposed
+//                     (MN-major), B = P, O (fp32) accumulated in tensor memory;
+//   warps 4..7        softmax (softmax_role): one tensor-memory load gives a token's HC
+//                     scores; the running max moves only when a score exceeds it by more
+//                     than 2^8 (one reducing barrier per page decides), in which case O
+//                     is rescaled before the next PV; P goes to shared memory (three
+//                     buffers) as the fp16 B operand.
+// Every kernel here is launched as a programmatic dependent of the previous one in the
+// stream and waits (griddepcontrol.wait) before it reads an input.
 // Kernel B (rolaq_decode_merge): log-sum-exp merge of the per-item partials.
 //
 // Fused append (one new token per request at position L - 1, the per-step write of a
