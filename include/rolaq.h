@@ -27,7 +27,11 @@
  *   - All pointers named *_dev are device pointers owned by the caller; the library
  *     never allocates, frees or keeps them.  Host pointers are read during the call only.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Work is
- *     enqueued asynchronously; the call returns once the kernels are launched.
+ *     enqueued asynchronously; the call returns once the kernels are launched.  The
+ *     decode, write-path and projection kernels are launched as programmatic dependents
+ *     of the previous work in the stream and wait for its completion before they read or
+ *     write memory, so stream order holds as for ordinary launches; only their start-up
+ *     overlaps the previous kernel's end.
  *   - Return value: ROLAQ_OK (0) or a negative ROLAQ_E* code.  Argument errors are
  *     detected on the host before anything is launched.  Errors that only the device can
  *     see (a page-table entry outside the pool) set bits in a device status word, skip
