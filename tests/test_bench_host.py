@@ -32,3 +32,19 @@ def test_sweep_unpackers_read_the_page_format():
 def test_sweep_taus_include_the_reference_threshold():
     assert bench.LLOYD_MAX_TAU in bench.SWEEP_TAUS
     assert abs(O.lloyd_max_threshold() - bench.LLOYD_MAX_TAU) < 1e-3
+
+
+def test_packed_host_buffers_round_trip():
+    """The end-to-end leg moves each step's inputs and outputs as one packed buffer: every
+    segment starts 256-byte aligned and reads back the tensor written into it."""
+    import torch
+    src = [torch.randn(4, 512).to(torch.bfloat16), torch.randn(4, 64).to(torch.bfloat16),
+           torch.randn(4, 16, 512).to(torch.bfloat16), torch.randn(4, 16), torch.randn(3)]
+    offs, total = bench.pack_offsets([(tuple(t.shape), t.dtype) for t in src])
+    assert all(o % 256 == 0 for o, _, _, _ in offs)
+    assert total >= sum(t.numel() * t.element_size() for t in src)
+    buf = torch.zeros(total, dtype=torch.uint8)
+    for v, t in zip(bench.pack_views(buf, offs), src):
+        v.copy_(t)
+    for v, t in zip(bench.pack_views(buf.clone(), offs), src):
+        assert torch.equal(v, t)
